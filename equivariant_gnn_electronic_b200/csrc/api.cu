@@ -1,0 +1,319 @@
+// Host side of the C ABI declared in include/egnn.h: argument checks, parameter
+// packing, Clebsch-Gordan tables, dispatch to the kernels.
+#include <math.h>
+#include <string.h>
+
+#include <complex>
+#include <vector>
+
+#include "common.cuh"
+#include "so2_params.cuh"
+
+size_t egnn_graph_workspace_bytes(int32_t n_atoms);   // graph.cu
+
+namespace {
+
+size_t dtype_size(int dt) { return dt == EGNN_BF16 ? 2 : 4; }
+
+egnn_status check_desc(const egnn_layer_desc* d) {
+  if (!d) return EGNN_ERR_INVALID_ARG;
+  if (d->dtype != EGNN_FP32 && d->dtype != EGNN_BF16) return EGNN_ERR_UNSUPPORTED;
+  if (d->lmax < 0 || d->lmax > 6 || d->mmax < 0 || d->mmax > 2 || d->mmax > d->lmax) return EGNN_ERR_UNSUPPORTED;
+  if (d->channels < 1 || d->channels > 128 || d->heads < 1 || d->heads > 16) return EGNN_ERR_UNSUPPORTED;
+  if (d->channels % d->heads) return EGNN_ERR_UNSUPPORTED;
+  if (d->n_rbf < 2 || d->n_rbf > 64) return EGNN_ERR_UNSUPPORTED;
+  if (!(d->rcut > 0.f)) return EGNN_ERR_INVALID_ARG;
+  return EGNN_OK;
+}
+
+egnn_status check_graph(const egnn_graph* g, const egnn_layer_desc* d) {
+  if (!g || !g->row_ptr || !g->status || g->n_atoms < 1) return EGNN_ERR_INVALID_ARG;
+  if (g->n_edges < 0 || g->n_edges > g->capacity) return EGNN_ERR_INVALID_ARG;
+  if (g->n_edges > 0 && (!g->src || !g->dist || !g->wigner)) return EGNN_ERR_INVALID_ARG;
+  if (g->lmax != d->lmax || g->mmax != d->mmax) return EGNN_ERR_INVALID_ARG;
+  return EGNN_OK;
+}
+
+void fill_params(So2Params& P, const egnn_graph* g, const egnn_layer_desc* d) {
+  memset(&P, 0, sizeof(P));
+  P.n_atoms = g->n_atoms;
+  P.n_edges = g->n_edges;
+  P.lmax = d->lmax;
+  P.mmax = d->mmax;
+  P.C = d->channels;
+  P.H = d->heads;
+  P.K = d->n_rbf;
+  P.L = d->lmax + 1;
+  P.L2 = P.L * P.L;
+  P.wfl = egnn_wigner_floats(d->lmax, d->mmax);
+  P.dtype = d->dtype;
+  P.rcut = d->rcut;
+  P.row_ptr = g->row_ptr;
+  P.src = g->src;
+  P.dist = g->dist;
+  P.wig = g->wigner;
+  P.status = g->status;
+  int r = 0;
+  for (int l = 0; l <= d->lmax; ++l) {
+    int ml = l < d->mmax ? l : d->mmax;
+    P.woff[l] = egnn_wig_off(l, d->mmax);
+    P.row0[l] = r + ml;
+    for (int m = -ml; m <= ml; ++m) {
+      P.row_l[r] = l;
+      P.row_m[r] = m;
+      ++r;
+    }
+    for (int m = -l; m <= l; ++m) P.coef_l[l * l + l + m] = l;
+  }
+  P.nrows = r;
+}
+
+// Carves the packed weight buffer (order documented in egnn.h); returns elements used.
+size_t carve_so2(So2Weights& W, const char* base, const egnn_layer_desc* d, bool attention) {
+  const size_t es = dtype_size(d->dtype);
+  const size_t L = d->lmax + 1, C = d->channels, K = d->n_rbf;
+  size_t o = 0;
+  auto take = [&](size_t n) { const void* p = base + o * es; o += n; return p; };
+  memset(&W, 0, sizeof(W));
+  W.W1 = take(C * K);
+  W.b1 = take(C);
+  W.W2 = take(L * 2 * C * C);
+  W.b2 = take(L * 2 * C);
+  W.W0 = take(L * C * L * 2 * C);
+  for (int m = 1; m <= d->mmax; ++m) {
+    size_t nm = L - m;
+    W.Wm[m - 1][0] = take(nm * C * nm * 2 * C);
+    W.Wm[m - 1][1] = take(nm * C * nm * 2 * C);
+  }
+  if (attention) {
+    W.A = take(d->heads * L * C);
+    W.bA = take(d->heads);
+  }
+  return o;
+}
+
+// ---------------- Clebsch-Gordan tables (library side) ----------------
+// Complex coefficients <j1 m1 j2 m2 | J M> by Racah's closed formula, then the
+// unitary change to the real basis of egnn.h (real_m = sum_mu U[m][mu] Y^mu,
+// Y^mu with the Condon-Shortley phase):  C_real = (U_la (x) U_lb) C U_L^dagger.
+// The result is real up to one global phase, removed before the sign rule
+// (first non-zero entry of column M = -L positive).
+double fact(int n) {
+  double r = 1;
+  for (int i = 2; i <= n; ++i) r *= i;
+  return r;
+}
+
+double cg_complex(int j1, int m1, int j2, int m2, int J, int M) {
+  if (m1 + m2 != M || abs(m1) > j1 || abs(m2) > j2 || abs(M) > J) return 0.0;
+  double pre = sqrt((2 * J + 1) * fact(J + j1 - j2) * fact(J - j1 + j2) * fact(j1 + j2 - J) /
+                    fact(j1 + j2 + J + 1));
+  pre *= sqrt(fact(J + M) * fact(J - M) * fact(j1 - m1) * fact(j1 + m1) * fact(j2 - m2) * fact(j2 + m2));
+  double s = 0.0;
+  for (int k = 0; k <= j1 + j2 + J; ++k) {
+    int a[6] = {k, j1 + j2 - J - k, j1 - m1 - k, j2 + m2 - k, J - j2 + m1 + k, J - j1 - m2 + k};
+    bool ok = true;
+    double den = 1.0;
+    for (int t = 0; t < 6; ++t) {
+      if (a[t] < 0) ok = false;
+      else den *= fact(a[t]);
+    }
+    if (ok) s += ((k & 1) ? -1.0 : 1.0) / den;
+  }
+  return pre * s;
+}
+
+std::complex<double> real_from_complex(int m, int mu) {
+  const double r = 1.0 / sqrt(2.0);
+  if (m == 0) return mu == 0 ? 1.0 : 0.0;
+  if (m > 0) {
+    if (mu == m) return ((m & 1) ? -r : r);
+    if (mu == -m) return r;
+    return 0.0;
+  }
+  int am = -m;
+  if (mu == am) return std::complex<double>(0.0, (am & 1) ? r : -r);
+  if (mu == -am) return std::complex<double>(0.0, r);
+  return 0.0;
+}
+
+void real_cg(int la, int lb, int L, std::vector<float>& out) {
+  int na = 2 * la + 1, nb = 2 * lb + 1, nl = 2 * L + 1;
+  std::vector<std::complex<double>> C(na * nb * nl);
+  for (int ma = -la; ma <= la; ++ma)
+    for (int mb = -lb; mb <= lb; ++mb)
+      for (int m = -L; m <= L; ++m) {
+        std::complex<double> s = 0.0;
+        for (int ua = -la; ua <= la; ++ua) {
+          std::complex<double> fa = real_from_complex(ma, ua);
+          if (fa == 0.0) continue;
+          for (int ub = -lb; ub <= lb; ++ub) {
+            std::complex<double> fb = real_from_complex(mb, ub);
+            if (fb == 0.0 || abs(ua + ub) > L) continue;
+            s += fa * fb * cg_complex(la, ua, lb, ub, L, ua + ub) * std::conj(real_from_complex(m, ua + ub));
+          }
+        }
+        C[((ma + la) * nb + (mb + lb)) * nl + (m + L)] = s;
+      }
+  double nr = 0, ni = 0;
+  for (auto& c : C) {
+    nr += c.real() * c.real();
+    ni += c.imag() * c.imag();
+  }
+  std::vector<double> R(C.size());
+  for (size_t i = 0; i < C.size(); ++i) R[i] = nr >= ni ? C[i].real() : C[i].imag();
+  for (int r = 0; r < na * nb; ++r) {
+    double v = R[(size_t)r * nl];
+    if (fabs(v) > 1e-9) {
+      if (v < 0)
+        for (auto& x : R) x = -x;
+      break;
+    }
+  }
+  for (double x : R) out.push_back((float)x);
+}
+
+}  // namespace
+
+extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* desc, int32_t n_atoms,
+                                       int64_t n_edges) {
+  (void)n_edges;
+  switch (which) {
+    case EGNN_WS_BUILD_GRAPH:
+      return egnn_graph_workspace_bytes(n_atoms);
+    case EGNN_WS_LAYER:
+      return 256;
+    case EGNN_WS_HAMILTONIAN:
+      return 64 * 1024;
+    default:
+      return 0;
+  }
+  (void)desc;
+}
+
+extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_desc* desc,
+                                          const void* weights, const void* node_in, void* node_out,
+                                          void* workspace, size_t ws_bytes, void* cuda_stream) {
+  egnn_status s = check_desc(desc);
+  if (s != EGNN_OK) return s;
+  if ((s = check_graph(g, desc)) != EGNN_OK) return s;
+  if (!weights || !node_in || !node_out || node_in == node_out) return EGNN_ERR_INVALID_ARG;
+  (void)workspace;
+  (void)ws_bytes;
+  cudaStream_t st = (cudaStream_t)cuda_stream;
+  So2Params P;
+  fill_params(P, g, desc);
+  P.node_in = node_in;
+  P.node_out = node_out;
+  So2Weights W;
+  carve_so2(W, (const char*)weights, desc, true);
+  P.te = so2_simt_pick_te(P, 0);
+  if (P.te < 1) return EGNN_ERR_UNSUPPORTED;
+  EGNN_CUDA_TRY(launch_layer_simt(P, W, st));
+  return EGNN_OK;
+}
+
+extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_layer_desc* desc,
+                                               const void* head_weights, const int32_t* shell_l,
+                                               int32_t n_shells, const void* node_emb, float* blocks,
+                                               void* workspace, size_t ws_bytes, void* cuda_stream) {
+  egnn_status s = check_desc(desc);
+  if (s != EGNN_OK) return s;
+  if ((s = check_graph(g, desc)) != EGNN_OK) return s;
+  if (!head_weights || !shell_l || !node_emb || (!blocks && g->n_edges > 0)) return EGNN_ERR_INVALID_ARG;
+  if (n_shells < 1 || n_shells > 16) return EGNN_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < egnn_workspace_bytes(EGNN_WS_HAMILTONIAN, desc, g->n_atoms, g->n_edges))
+    return EGNN_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)cuda_stream;
+  HeadTables T;
+  memset(&T, 0, sizeof(T));
+  T.n_shells = n_shells;
+  int o = 0;
+  for (int a = 0; a < n_shells; ++a) {
+    int l = shell_l[a];
+    if (l < 0 || l > 3) return EGNN_ERR_UNSUPPORTED;
+    T.shell_l[a] = l;
+    T.shell_off[a] = o;
+    if (o + 2 * l + 1 > 32) return EGNN_ERR_UNSUPPORTED;
+    for (int i = 0; i < 2 * l + 1; ++i) T.orb_shell[o + i] = a;
+    o += 2 * l + 1;
+    for (int b = 0; b < a; ++b)
+      if (shell_l[b] + l > desc->lmax) return EGNN_ERR_UNSUPPORTED;
+    if (2 * l > desc->lmax) return EGNN_ERR_UNSUPPORTED;
+  }
+  T.shell_off[n_shells] = o;
+  T.n_orb = o;
+  // label multiplicities and k index per (a, b, L): pairs lexicographic, a outer
+  std::vector<int> kidx(n_shells * n_shells * 8, 0);
+  int mult[8] = {0};
+  for (int a = 0; a < n_shells; ++a)
+    for (int b = 0; b < n_shells; ++b)
+      for (int Lc = abs(shell_l[a] - shell_l[b]); Lc <= shell_l[a] + shell_l[b]; ++Lc)
+        kidx[(a * n_shells + b) * 8 + Lc] = mult[Lc]++;
+  int lab = 0;
+  for (int Lc = 0; Lc <= desc->lmax; ++Lc) {
+    T.mult[Lc] = mult[Lc];
+    T.lab_off[Lc] = lab;
+    lab += (2 * Lc + 1) * mult[Lc];
+  }
+  for (int Lc = desc->lmax + 1; Lc < 8; ++Lc) T.lab_off[Lc] = lab;
+  T.n_lab = lab;
+  std::vector<float> cg;
+  for (int la = 0; la <= 3; ++la)
+    for (int lb = 0; lb <= 3; ++lb)
+      for (int Lc = abs(la - lb); Lc <= la + lb; ++Lc) {
+        T.cg_off[(la * 4 + lb) * 8 + Lc] = (int)cg.size();
+        real_cg(la, lb, Lc, cg);
+      }
+  size_t need = kidx.size() * sizeof(int) + cg.size() * sizeof(float) + 64;
+  if (ws_bytes < need) return EGNN_ERR_INVALID_ARG;
+  char* wsp = (char*)workspace;
+  EGNN_CUDA_TRY(cudaMemcpyAsync(wsp, kidx.data(), kidx.size() * sizeof(int), cudaMemcpyHostToDevice, st));
+  size_t off = (kidx.size() * sizeof(int) + 15) & ~(size_t)15;
+  EGNN_CUDA_TRY(cudaMemcpyAsync(wsp + off, cg.data(), cg.size() * sizeof(float), cudaMemcpyHostToDevice, st));
+  T.kidx = (const int*)wsp;
+  T.cg = (const float*)(wsp + off);
+
+  So2Params P;
+  fill_params(P, g, desc);
+  if (2 * P.nrows < P.L2) return EGNN_ERR_UNSUPPORTED;
+  P.node_in = node_emb;
+  P.blocks = blocks;
+  So2Weights W;
+  size_t used = carve_so2(W, (const char*)head_weights, desc, false);
+  const size_t es = dtype_size(desc->dtype);
+  for (int Lc = 0; Lc <= desc->lmax; ++Lc) {
+    if (mult[Lc]) {
+      W.U[Lc] = (const char*)head_weights + used * es;
+      used += (size_t)mult[Lc] * desc->channels;
+    }
+  }
+  P.te = so2_simt_pick_te(P, T.n_lab);
+  if (P.te < 1) return EGNN_ERR_UNSUPPORTED;
+  if (g->n_edges == 0) return EGNN_OK;
+  EGNN_CUDA_TRY(launch_head_simt(P, W, T, st));
+  // the tables live in `workspace`: keep them until the kernel has read them
+  return EGNN_OK;
+}
+
+extern "C" egnn_status egnn_read_status(const egnn_graph* g, int32_t* code, void* cuda_stream) {
+  if (!g || !g->status) return EGNN_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaStream_t st = (cudaStream_t)cuda_stream;
+  EGNN_CUDA_TRY(cudaMemcpyAsync(&v, g->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  EGNN_CUDA_TRY(cudaStreamSynchronize(st));
+  if (code) *code = v;
+  return v ? EGNN_ERR_DEVICE_CHECK : EGNN_OK;
+}
+
+extern "C" const char* egnn_status_string(egnn_status s) {
+  switch (s) {
+    case EGNN_OK: return "ok";
+    case EGNN_ERR_INVALID_ARG: return "invalid argument";
+    case EGNN_ERR_CAPACITY: return "graph capacity too small (n_edges holds the required count)";
+    case EGNN_ERR_UNSUPPORTED: return "unsupported size, dtype or template";
+    case EGNN_ERR_CUDA: return "CUDA runtime error";
+    case EGNN_ERR_DEVICE_CHECK: return "device-side check failed (see status word)";
+  }
+  return "unknown status";
+}

@@ -1,0 +1,147 @@
+"""GPU eSCN layer and Hamiltonian head against the oracle.
+
+Small cells are compared element by element over every atom; the full-size
+workloads on a seeded sample of destination atoms (the layer is local to each
+destination atom, so a sampled atom's output is exact, not statistical).
+Tolerances: fp32 1e-4, bf16 storage / fp32 accumulation 2e-2, as max relative
+error max|gpu - ref| / max|ref|, applied to the output and to the update
+out - n_d separately."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_helpers import TOL, cell, gpu_graph, oracle_graph, rel_err, sample_atoms, to_dev
+from oracle import head as ohead
+from oracle import layer as olayer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def egnn():
+    from equivariant_gnn_electronic_b200 import egnn
+    return egnn
+
+
+def _kw(w):
+    return dict(lmax=w.lmax, mmax=w.mmax, rcut=w.rcut, n_rbf=w.n_rbf)
+
+
+def run_layer(egnn, name, w, seed=0, n_atoms=None, atoms=None, bias_std=0.0):
+    pos, _, box = cell(name, seed, n_atoms)
+    g = gpu_graph(egnn, name, seed, n_atoms, lmax=w.lmax, mmax=w.mmax)
+    desc = egnn.desc_for(w)
+    dt = egnn.torch_dtype(desc)
+    n = synth.make_embeddings(w, len(pos), seed)
+    W = synth.make_layer_weights(w, seed, bias_std=bias_std)
+    out = egnn.layer_forward(g, desc, egnn.pack_weights(W, desc), to_dev(n, dt))
+    torch.cuda.synchronize()
+    assert g.read_status() == 0
+    got = out.float().cpu().numpy().astype(np.float64)
+    rp, src, sh = oracle_graph(name, seed, n_atoms)
+    sel = np.arange(len(pos)) if atoms is None else atoms
+    ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads, atoms=sel)
+    return got[sel], ref, n[sel]
+
+
+def check(got, ref, nd, tol):
+    """Output within tol; the update out - n_d too (bf16: the output's own rounding
+    is relative to |out|, not to the smaller update, hence 2.5x there)."""
+    e_out = rel_err(got, ref)
+    e_upd = rel_err(got - nd, ref - nd)
+    assert e_out < tol, e_out
+    assert e_upd < (tol if tol < 1e-3 else 2.5 * tol), e_upd
+
+
+def test_layer_tiny_fp32_every_atom(egnn):
+    w = synth.WORKLOADS["tiny"]
+    got, ref, nd = run_layer(egnn, "tiny", w, bias_std=0.2)
+    check(got, ref, nd, TOL["fp32"])
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_layer_tiny_more_seeds(egnn, seed):
+    w = synth.WORKLOADS["tiny"]
+    got, ref, nd = run_layer(egnn, "tiny", w, seed=seed)
+    check(got, ref, nd, TOL["fp32"])
+
+
+def test_layer_small_bf16_every_atom(egnn):
+    # 300-atom HfO2-density cell, full C=128, lmax 4: many chunks per atom
+    w = synth.WORKLOADS["hfo2_3000"]
+    got, ref, nd = run_layer(egnn, "hfo2_3000", w, n_atoms=300, bias_std=0.1)
+    check(got, ref, nd, TOL["bf16"])
+
+
+@pytest.mark.parametrize("name", ["hfo2_3000", "gst_8064", "mixed_12000"])
+def test_layer_full_size_sampled(egnn, name):
+    w = synth.WORKLOADS[name]
+    pos, _, _ = cell(name)
+    atoms = np.concatenate([[0, len(pos) - 1], sample_atoms(len(pos), 30, 3)])
+    got, ref, nd = run_layer(egnn, name, w, atoms=np.unique(atoms))
+    check(got, ref, nd, TOL["bf16"])
+
+
+def test_layer_isolated_atom_keeps_embedding(egnn):
+    w = synth.WORKLOADS["tiny"]
+    box = np.array([100.0, 100.0, 100.0])
+    pos = np.array([[1.0, 1.0, 1.0], [50.0, 50.0, 50.0], [52.0, 50.0, 50.0], [50.0, 53.0, 50.0]])
+    g = gpu_graph(egnn, "tiny", pos=pos, box=box)
+    desc = egnn.desc_for(w)
+    n = np.random.default_rng(0).standard_normal((4, 9, 16))
+    W = synth.make_layer_weights(w, 0)
+    out = egnn.layer_forward(g, desc, egnn.pack_weights(W, desc), to_dev(n, torch.float32)).cpu().numpy()
+    np.testing.assert_array_equal(out[0], n[0].astype(np.float32))
+    from oracle import graph as og
+    rp, src, sh = og.neighbour_list_bruteforce(pos, box, w.rcut)
+    ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
+    assert rel_err(out, ref) < TOL["fp32"]
+
+
+def test_layer_is_deterministic(egnn):
+    w = synth.WORKLOADS["hfo2_3000"]
+    pos, species, box = cell("hfo2_3000", 0, 300)
+    g = gpu_graph(egnn, "hfo2_3000", 0, 300)
+    desc = egnn.desc_for(w)
+    n = to_dev(synth.make_embeddings(w, len(pos), 0), torch.bfloat16)
+    Wp = egnn.pack_weights(synth.make_layer_weights(w, 0), desc)
+    a = egnn.layer_forward(g, desc, Wp, n).clone()
+    b = egnn.layer_forward(g, desc, Wp, n)
+    assert torch.equal(a, b)
+
+
+def run_head(egnn, name, w, seed=0, n_atoms=None, atoms=None, bias_std=0.0, shells=None):
+    shells = w.shells if shells is None else shells
+    pos, _, box = cell(name, seed, n_atoms)
+    g = gpu_graph(egnn, name, seed, n_atoms, lmax=w.lmax, mmax=w.mmax)
+    desc = egnn.desc_for(w)
+    dt = egnn.torch_dtype(desc)
+    n = synth.make_embeddings(w, len(pos), seed)
+    HW = synth.make_head_weights(w, seed, bias_std=bias_std, shells=shells)
+    blocks = egnn.hamiltonian_blocks(g, desc, egnn.pack_weights(HW, desc, attention=False), shells,
+                                     to_dev(n, dt))
+    torch.cuda.synchronize()
+    assert g.read_status() == 0
+    got = blocks.cpu().numpy().astype(np.float64)
+    rp, src, sh = oracle_graph(name, seed, n_atoms)
+    sel = np.arange(len(pos)) if atoms is None else atoms
+    ref = ohead.hamiltonian_blocks(pos, box, rp, src, sh, n, HW, shells, **_kw(w), atoms=sel)
+    idx = np.concatenate([np.arange(rp[a], rp[a + 1]) for a in sel])
+    return got[idx], ref
+
+
+def test_head_tiny_fp32_every_edge(egnn):
+    w = synth.WORKLOADS["tiny"]
+    got, ref = run_head(egnn, "tiny", w, bias_std=0.2)
+    assert rel_err(got, ref) < TOL["fp32"]
+
+
+@pytest.mark.parametrize("name", ["gst_8064", "mixed_12000"])
+def test_head_full_size_sampled(egnn, name):
+    w = synth.WORKLOADS[name]
+    pos, _, _ = cell(name)
+    got, ref = run_head(egnn, name, w, atoms=sample_atoms(len(pos), 4, 5))
+    assert rel_err(got, ref) < TOL["bf16"]

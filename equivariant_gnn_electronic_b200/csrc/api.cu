@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "so2_params.cuh"
+#include "so2_tc.cuh"
 
 size_t egnn_graph_workspace_bytes(int32_t n_atoms);   // graph.cu
 
@@ -90,6 +91,67 @@ size_t carve_so2(So2Weights& W, const char* base, const egnn_layer_desc* d, bool
     W.bA = take(d->heads);
   }
   return o;
+}
+
+// ---------------- tensor-core layer plan ----------------
+bool tc_eligible(const egnn_layer_desc* d) {
+  return d->dtype == EGNN_BF16 && d->channels == 128 && d->lmax >= 1 && d->lmax <= 6 && d->mmax <= 2 &&
+         d->heads <= 16 && 128 % d->heads == 0;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Pass list: radial-gate passes, then the SO(2) blocks |m| = 0..mmax, each block's
+// output rows split into accumulators of at most 512 TMEM columns.
+void tc_plan(const egnn_layer_desc* d, TcParams& P) {
+  const int L = d->lmax + 1, C = d->channels;
+  P.npass = 0;
+  long long boff = 0;
+  auto add = [&](int kind, int block, int ntot, int nk) {
+    for (int off = 0; off < ntot; off += 512) {
+      TcPass& q = P.pass[P.npass++];
+      q.kind = kind;
+      q.block = block;
+      q.n = ntot - off < 512 ? ntot - off : 512;
+      q.n_off = off;
+      q.nk = nk;
+      q.last_of_kind = 0;
+      q.boff = boff;
+      boff += (long long)q.n * nk * 128;
+    }
+    P.pass[P.npass - 1].last_of_kind = 1;
+  };
+  add(0, 0, L * 2 * C, C / 64);
+  int ycol = 0;
+  for (int b = 0; b <= d->mmax; ++b) {
+    int nb = b == 0 ? L * C : 2 * (L - b) * C;
+    int kb = b == 0 ? L * 2 * C : 2 * (L - b) * 2 * C;
+    P.ybase[b] = ycol;
+    ycol += nb;
+    add(1, b, nb, kb / 64);
+    if (b > 0) P.pass[P.npass - 1].last_of_kind = 0;
+  }
+  P.ncols_y = ycol;
+  P.gcols = L * 2 * C;
+  P.wprep_bytes = boff;
+}
+
+struct TcWorkspace {
+  size_t wprep, gate, y, logits, total;
+};
+
+TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges) {
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  tc_plan(d, P);
+  TcWorkspace w;
+  size_t E = n_edges > 0 ? (size_t)n_edges : 0;
+  w.wprep = 0;
+  w.gate = align_up((size_t)P.wprep_bytes, 1024);
+  w.y = w.gate + align_up((size_t)kTcMaxGrid * 128 * P.gcols * 2, 1024);
+  w.logits = w.y + align_up(E * P.ncols_y * 2, 1024);
+  w.total = w.logits + align_up(E * d->heads * 4, 1024) + 1024;
+  return w;
 }
 
 // ---------------- Clebsch-Gordan tables (library side) ----------------
@@ -182,6 +244,7 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
     case EGNN_WS_BUILD_GRAPH:
       return egnn_graph_workspace_bytes(n_atoms);
     case EGNN_WS_LAYER:
+      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc)) return tc_workspace(desc, n_edges).total;
       return 256;
     case EGNN_WS_HAMILTONIAN:
       return 64 * 1024;
@@ -198,9 +261,58 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
   if (s != EGNN_OK) return s;
   if ((s = check_graph(g, desc)) != EGNN_OK) return s;
   if (!weights || !node_in || !node_out || node_in == node_out) return EGNN_ERR_INVALID_ARG;
-  (void)workspace;
-  (void)ws_bytes;
   cudaStream_t st = (cudaStream_t)cuda_stream;
+  if (tc_eligible(desc)) {
+    TcWorkspace wl = tc_workspace(desc, g->n_edges);
+    if (!workspace || ws_bytes < wl.total) return EGNN_ERR_INVALID_ARG;
+    uint8_t* ws = (uint8_t*)(((uintptr_t)workspace + 1023) & ~(uintptr_t)1023);
+    if ((size_t)(ws - (uint8_t*)workspace) + wl.total - 1024 > ws_bytes) return EGNN_ERR_INVALID_ARG;
+    TcParams T;
+    memset(&T, 0, sizeof(T));
+    tc_plan(desc, T);
+    T.n_atoms = g->n_atoms;
+    T.n_edges = g->n_edges;
+    T.n_tiles = (int)((g->n_edges + 127) / 128);
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    T.grid = nsm < kTcMaxGrid ? nsm : kTcMaxGrid;
+    if (T.grid > T.n_tiles) T.grid = T.n_tiles > 0 ? T.n_tiles : 1;
+    T.lmax = desc->lmax;
+    T.mmax = desc->mmax;
+    T.C = desc->channels;
+    T.H = desc->heads;
+    T.K = desc->n_rbf;
+    T.L = desc->lmax + 1;
+    T.L2 = T.L * T.L;
+    T.wfl = egnn_wigner_floats(desc->lmax, desc->mmax);
+    T.rcut = desc->rcut;
+    T.row_ptr = g->row_ptr;
+    T.src = g->src;
+    T.dist = g->dist;
+    T.wig = g->wigner;
+    T.status = g->status;
+    T.node_in = (const __nv_bfloat16*)node_in;
+    T.node_out = (__nv_bfloat16*)node_out;
+    for (int l = 0; l <= desc->lmax; ++l) T.woff[l] = egnn_wig_off(l, desc->mmax);
+    So2Weights W;
+    carve_so2(W, (const char*)weights, desc, true);
+    T.W1 = (const __nv_bfloat16*)W.W1;
+    T.b1 = (const __nv_bfloat16*)W.b1;
+    T.b2 = (const __nv_bfloat16*)W.b2;
+    T.A = (const __nv_bfloat16*)W.A;
+    T.bA = (const __nv_bfloat16*)W.bA;
+    T.wprep = ws + wl.wprep;
+    T.gate_scratch = (__nv_bfloat16*)(ws + wl.gate);
+    T.Y = (__nv_bfloat16*)(ws + wl.y);
+    T.logits = (float*)(ws + wl.logits);
+    TcWeights TW;
+    TW.W2 = (const __nv_bfloat16*)W.W2;
+    TW.W0 = (const __nv_bfloat16*)W.W0;
+    for (int m = 0; m < 2; ++m)
+      for (int k = 0; k < 2; ++k) TW.Wm[m][k] = (const __nv_bfloat16*)W.Wm[m][k];
+    EGNN_CUDA_TRY(launch_layer_tc(T, TW, st));
+    return EGNN_OK;
+  }
   So2Params P;
   fill_params(P, g, desc);
   P.node_in = node_in;

@@ -1,0 +1,51 @@
+// Launch parameters of the tensor-core eSCN layer (CUDA path only).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+// One GEMM pass over a 128-edge tile: D[128 x n] = A[128 x 64*nk] B[n x 64*nk]^T.
+struct TcPass {
+  int kind;          // 0 = radial gate (A = hidden layer), 1 = SO(2) block
+  int block;         // |m| of the SO(2) block
+  int n;             // accumulator columns (<= 512, multiple of 32)
+  int n_off;         // first output row of the block matrix covered by this pass
+  int nk;            // K chunks of 64
+  int last_of_kind;  // last gate pass / last pass of block 0
+  long long boff;    // byte offset of the pass's first B tile in the prepared image
+};
+
+struct TcParams {
+  int n_atoms;
+  long long n_edges;
+  int n_tiles, grid;
+  int lmax, mmax, C, H, K, L, L2, wfl, ncols_y, gcols;
+  float rcut;
+  const int32_t* row_ptr;
+  const int32_t* src;
+  const float* dist;
+  const float* wig;
+  const __nv_bfloat16* node_in;
+  __nv_bfloat16* node_out;
+  const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
+  const uint8_t* wprep;
+  long long wprep_bytes;
+  __nv_bfloat16* gate_scratch;   // [grid][128][gcols]
+  __nv_bfloat16* Y;              // [n_edges][ncols_y]
+  float* logits;                 // [n_edges][H]
+  int32_t* status;
+  int npass;
+  TcPass pass[16];
+  int woff[8];
+  int ybase[3];
+};
+
+struct TcWeights {
+  const __nv_bfloat16 *W2, *W0;
+  const __nv_bfloat16* Wm[2][2];
+};
+
+constexpr int kTcMaxGrid = 160;
+
+size_t so2_tc_smem_bytes();
+cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st);

@@ -418,3 +418,55 @@ extern "C" egnn_status egnn_build_graph(const double* pos, const int32_t* specie
   EGNN_CUDA_TRY(cudaGetLastError());
   return EGNN_OK;
 }
+
+// ---------------------------------------------------------------------------
+// egnn_build_graph_noalloc: the same graph build for callers that cannot hand the
+// library a device workspace.  Its scratch is a fixed array in this module's
+// device memory; every GPU that loads the library holds one copy until exit.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr int32_t kNoAllocMaxAtoms = 131072;
+// egnn_graph_workspace_bytes(n) needs 9n + 322 int32 words; round up generously.
+constexpr size_t kNoAllocScratchWords = 9 * (size_t)kNoAllocMaxAtoms + 1024;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchWords];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[128] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device.  The host-side name
+// is only a stand-in, so the address is looked up once per device (with that
+// device current) and cached.
+egnn_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EGNN_ERR_CUDA;
+  if (dev < 0 || dev >= 128) return EGNN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return EGNN_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return EGNN_OK;
+}
+
+}  // namespace
+
+extern "C" egnn_status egnn_build_graph_noalloc(const double* pos, const int32_t* species, int32_t n_atoms,
+                                                const double box[3], double rcut, int32_t lmax, int32_t mmax,
+                                                egnn_graph* g, void* cuda_stream) {
+  if (n_atoms > kNoAllocMaxAtoms) return EGNN_ERR_UNSUPPORTED;
+  if (!pos || !species || !box || !g || n_atoms < 1) return EGNN_ERR_INVALID_ARG;
+  size_t need = egnn_graph_workspace_bytes(n_atoms);
+  if (need > sizeof(int32_t) * kNoAllocScratchWords) return EGNN_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  egnn_status s = noalloc_scratch(&scratch);
+  if (s != EGNN_OK) return s;
+  return egnn_build_graph(pos, species, n_atoms, box, rcut, lmax, mmax, g, scratch,
+                          sizeof(int32_t) * kNoAllocScratchWords, cuda_stream);
+}

@@ -22,7 +22,7 @@ EGNN_WS_BUILD_GRAPH, EGNN_WS_LAYER, EGNN_WS_HAMILTONIAN = 0, 1, 2
 
 EXPORTED = (
     "egnn_wigner_floats", "egnn_workspace_bytes", "egnn_build_graph", "egnn_layer_forward",
-    "egnn_hamiltonian_blocks", "egnn_read_status", "egnn_status_string",
+    "egnn_hamiltonian_blocks", "egnn_read_status", "egnn_status_string", "egnn_build_graph_noalloc",
 )
 
 
@@ -57,6 +57,9 @@ def _load():
     lib.egnn_build_graph.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_double), ctypes.c_double,
                                      i32, i32, ctypes.POINTER(GraphStruct), vp, sz, vp]
     lib.egnn_build_graph.restype = i32
+    lib.egnn_build_graph_noalloc.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_double), ctypes.c_double,
+                                             i32, i32, ctypes.POINTER(GraphStruct), vp]
+    lib.egnn_build_graph_noalloc.restype = i32
     lib.egnn_layer_forward.argtypes = [ctypes.POINTER(GraphStruct), ctypes.POINTER(LayerDesc), vp, vp,
                                        vp, vp, sz, vp]
     lib.egnn_layer_forward.restype = i32
@@ -183,6 +186,15 @@ def build_graph(pos: torch.Tensor, species: torch.Tensor, box: Sequence[float], 
         _check(code, "egnn_build_graph")
         return graph
     raise EgnnError(EGNN_ERR_CAPACITY, "egnn_build_graph")
+
+
+def build_graph_noalloc(pos: torch.Tensor, species: torch.Tensor, box: Sequence[float], rcut: float,
+                        lmax: int, mmax: int, graph: Graph, stream=None) -> int:
+    """egnn_build_graph_noalloc into an existing Graph (no workspace); returns the status code."""
+    assert pos.dtype == torch.float64 and pos.is_cuda and pos.is_contiguous()
+    boxarr = (ctypes.c_double * 3)(*[float(b) for b in box])
+    return int(lib.egnn_build_graph_noalloc(_ptr(pos), _ptr(species), pos.shape[0], boxarr, float(rcut),
+                                            lmax, mmax, ctypes.byref(graph.s), _stream(stream)))
 
 
 def layer_forward(graph: Graph, desc: LayerDesc, weights: torch.Tensor, node_in: torch.Tensor,

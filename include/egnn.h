@@ -12,7 +12,8 @@
  * Conventions shared by every call
  *   - Every pointer named "device" is CUDA device memory owned by the caller.
  *     The library allocates nothing (no cudaMalloc, no library allocator): all
- *     scratch comes from the caller's `workspace`, sized by egnn_workspace_bytes.
+ *     scratch comes from the caller's `workspace`, sized by egnn_workspace_bytes,
+ *     except in egnn_build_graph_noalloc (a fixed array in the library's module).
  *   - Work is launched on `cuda_stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Calls are asynchronous unless stated otherwise.
  *   - Host-checkable errors (null pointers, unsupported sizes, workspace too
@@ -109,6 +110,28 @@ size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* desc, int32_t 
 egnn_status egnn_build_graph(const double* pos, const int32_t* species, int32_t n_atoms,
                              const double box[3], double rcut, int32_t lmax, int32_t mmax,
                              egnn_graph* g, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * egnn_build_graph_noalloc -- egnn_build_graph without a caller-supplied workspace.
+ * The pages have no counterpart to this call; it exists for callers that cannot
+ * obtain device memory for a workspace, for example a component that only
+ * receives device pointers from its host application and may not call
+ * cudaMalloc itself, or a loop that forbids allocation after start-up.  It makes
+ * no allocation of any kind: its scratch is a fixed array of about 4.7 MB in the
+ * library's device memory, one copy on every GPU that loads the library, held
+ * until the process exits.
+ * Arguments, outputs and errors are those of egnn_build_graph, plus:
+ *   n_atoms above 131072 returns EGNN_ERR_UNSUPPORTED before any work;
+ *   the first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.
+ * All calls share the one array (whatever stream they use) and the kernels clear
+ * what must start at zero, so calls that overlap on the GPU race: order them, for
+ * example on one stream.
+ */
+egnn_status egnn_build_graph_noalloc(const double* pos, const int32_t* species, int32_t n_atoms,
+                                     const double box[3], double rcut, int32_t lmax, int32_t mmax,
+                                     egnn_graph* g, void* cuda_stream);
 
 /*
  * egnn_layer_forward -- one eSCN message-passing layer in the incoming-edge layout.

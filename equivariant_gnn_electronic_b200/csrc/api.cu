@@ -154,6 +154,56 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges) {
   return w;
 }
 
+// Fills the tensor-core launch parameters for graph g, weights W and a 1024-aligned
+// workspace; returns false if the workspace is too small.
+bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_desc* desc, const So2Weights& W,
+             const void* node_in, void* node_out, uint8_t* ws, int with_logits) {
+  TcWorkspace wl = tc_workspace(desc, g->n_edges);
+  memset(&T, 0, sizeof(T));
+  tc_plan(desc, T);
+  T.n_atoms = g->n_atoms;
+  T.n_edges = g->n_edges;
+  T.n_tiles = (int)((g->n_edges + 127) / 128);
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  T.grid = nsm < kTcMaxGrid ? nsm : kTcMaxGrid;
+  if (T.grid > T.n_tiles) T.grid = T.n_tiles > 0 ? T.n_tiles : 1;
+  T.lmax = desc->lmax;
+  T.mmax = desc->mmax;
+  T.C = desc->channels;
+  T.H = desc->heads;
+  T.K = desc->n_rbf;
+  T.L = desc->lmax + 1;
+  T.L2 = T.L * T.L;
+  T.wfl = egnn_wigner_floats(desc->lmax, desc->mmax);
+  T.rcut = desc->rcut;
+  T.row_ptr = g->row_ptr;
+  T.src = g->src;
+  T.dist = g->dist;
+  T.wig = g->wigner;
+  T.status = g->status;
+  T.with_logits = with_logits;
+  T.node_in = (const __nv_bfloat16*)node_in;
+  T.node_out = (__nv_bfloat16*)node_out;
+  for (int l = 0; l <= desc->lmax; ++l) T.woff[l] = egnn_wig_off(l, desc->mmax);
+  T.W1 = (const __nv_bfloat16*)W.W1;
+  T.b1 = (const __nv_bfloat16*)W.b1;
+  T.b2 = (const __nv_bfloat16*)W.b2;
+  T.A = (const __nv_bfloat16*)W.A;
+  T.bA = (const __nv_bfloat16*)W.bA;
+  T.wprep = ws + wl.wprep;
+  T.gate_scratch = (__nv_bfloat16*)(ws + wl.gate);
+  T.Y = (__nv_bfloat16*)(ws + wl.y);
+  T.logits = (float*)(ws + wl.logits);
+  TW.W2 = (const __nv_bfloat16*)W.W2;
+  TW.W0 = (const __nv_bfloat16*)W.W0;
+  for (int m = 0; m < 2; ++m)
+    for (int k = 0; k < 2; ++k) TW.Wm[m][k] = (const __nv_bfloat16*)W.Wm[m][k];
+  return true;
+}
+
+uint8_t* align1024(void* p) { return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023); }
+
 // ---------------- Clebsch-Gordan tables (library side) ----------------
 // Complex coefficients <j1 m1 j2 m2 | J M> by Racah's closed formula, then the
 // unitary change to the real basis of egnn.h (real_m = sum_mu U[m][mu] Y^mu,
@@ -247,6 +297,8 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc)) return tc_workspace(desc, n_edges).total;
       return 256;
     case EGNN_WS_HAMILTONIAN:
+      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
+        return tc_workspace(desc, n_edges).total + 64 * 1024;
       return 64 * 1024;
     default:
       return 0;
@@ -265,51 +317,12 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
   if (tc_eligible(desc)) {
     TcWorkspace wl = tc_workspace(desc, g->n_edges);
     if (!workspace || ws_bytes < wl.total) return EGNN_ERR_INVALID_ARG;
-    uint8_t* ws = (uint8_t*)(((uintptr_t)workspace + 1023) & ~(uintptr_t)1023);
-    if ((size_t)(ws - (uint8_t*)workspace) + wl.total - 1024 > ws_bytes) return EGNN_ERR_INVALID_ARG;
-    TcParams T;
-    memset(&T, 0, sizeof(T));
-    tc_plan(desc, T);
-    T.n_atoms = g->n_atoms;
-    T.n_edges = g->n_edges;
-    T.n_tiles = (int)((g->n_edges + 127) / 128);
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    T.grid = nsm < kTcMaxGrid ? nsm : kTcMaxGrid;
-    if (T.grid > T.n_tiles) T.grid = T.n_tiles > 0 ? T.n_tiles : 1;
-    T.lmax = desc->lmax;
-    T.mmax = desc->mmax;
-    T.C = desc->channels;
-    T.H = desc->heads;
-    T.K = desc->n_rbf;
-    T.L = desc->lmax + 1;
-    T.L2 = T.L * T.L;
-    T.wfl = egnn_wigner_floats(desc->lmax, desc->mmax);
-    T.rcut = desc->rcut;
-    T.row_ptr = g->row_ptr;
-    T.src = g->src;
-    T.dist = g->dist;
-    T.wig = g->wigner;
-    T.status = g->status;
-    T.node_in = (const __nv_bfloat16*)node_in;
-    T.node_out = (__nv_bfloat16*)node_out;
-    for (int l = 0; l <= desc->lmax; ++l) T.woff[l] = egnn_wig_off(l, desc->mmax);
+    uint8_t* ws = align1024(workspace);
     So2Weights W;
     carve_so2(W, (const char*)weights, desc, true);
-    T.W1 = (const __nv_bfloat16*)W.W1;
-    T.b1 = (const __nv_bfloat16*)W.b1;
-    T.b2 = (const __nv_bfloat16*)W.b2;
-    T.A = (const __nv_bfloat16*)W.A;
-    T.bA = (const __nv_bfloat16*)W.bA;
-    T.wprep = ws + wl.wprep;
-    T.gate_scratch = (__nv_bfloat16*)(ws + wl.gate);
-    T.Y = (__nv_bfloat16*)(ws + wl.y);
-    T.logits = (float*)(ws + wl.logits);
+    TcParams T;
     TcWeights TW;
-    TW.W2 = (const __nv_bfloat16*)W.W2;
-    TW.W0 = (const __nv_bfloat16*)W.W0;
-    for (int m = 0; m < 2; ++m)
-      for (int k = 0; k < 2; ++k) TW.Wm[m][k] = (const __nv_bfloat16*)W.Wm[m][k];
+    fill_tc(T, TW, g, desc, W, node_in, node_out, ws, 1);
     EGNN_CUDA_TRY(launch_layer_tc(T, TW, st));
     return EGNN_OK;
   }
@@ -377,20 +390,18 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
         T.cg_off[(la * 4 + lb) * 8 + Lc] = (int)cg.size();
         real_cg(la, lb, Lc, cg);
       }
-  size_t need = kidx.size() * sizeof(int) + cg.size() * sizeof(float) + 64;
+  const bool use_tc = tc_eligible(desc);
+  const size_t tc_bytes = use_tc ? tc_workspace(desc, g->n_edges).total : 0;
+  size_t need = tc_bytes + kidx.size() * sizeof(int) + cg.size() * sizeof(float) + 64;
   if (ws_bytes < need) return EGNN_ERR_INVALID_ARG;
-  char* wsp = (char*)workspace;
+  uint8_t* ws_tc = align1024(workspace);
+  char* wsp = use_tc ? (char*)(ws_tc + tc_bytes - 1024) : (char*)workspace;
   EGNN_CUDA_TRY(cudaMemcpyAsync(wsp, kidx.data(), kidx.size() * sizeof(int), cudaMemcpyHostToDevice, st));
   size_t off = (kidx.size() * sizeof(int) + 15) & ~(size_t)15;
   EGNN_CUDA_TRY(cudaMemcpyAsync(wsp + off, cg.data(), cg.size() * sizeof(float), cudaMemcpyHostToDevice, st));
   T.kidx = (const int*)wsp;
   T.cg = (const float*)(wsp + off);
 
-  So2Params P;
-  fill_params(P, g, desc);
-  if (2 * P.nrows < P.L2) return EGNN_ERR_UNSUPPORTED;
-  P.node_in = node_emb;
-  P.blocks = blocks;
   So2Weights W;
   size_t used = carve_so2(W, (const char*)head_weights, desc, false);
   const size_t es = dtype_size(desc->dtype);
@@ -400,6 +411,22 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
       used += (size_t)mult[Lc] * desc->channels;
     }
   }
+  if (use_tc) {
+    if (g->n_edges == 0) return EGNN_OK;
+    TcParams TP;
+    TcWeights TW;
+    fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, 0);
+    HeadUPtrs Up;
+    for (int Lc = 0; Lc < 8; ++Lc) Up.U[Lc] = (const __nv_bfloat16*)W.U[Lc];
+    if (head_tc_smem_bytes(TP, T.n_lab, 1) > 200 * 1024) return EGNN_ERR_UNSUPPORTED;
+    EGNN_CUDA_TRY(launch_head_tc(TP, TW, T, Up, blocks, st));
+    return EGNN_OK;
+  }
+  So2Params P;
+  fill_params(P, g, desc);
+  if (2 * P.nrows < P.L2) return EGNN_ERR_UNSUPPORTED;
+  P.node_in = node_emb;
+  P.blocks = blocks;
   P.te = so2_simt_pick_te(P, T.n_lab);
   if (P.te < 1) return EGNN_ERR_UNSUPPORTED;
   if (g->n_edges == 0) return EGNN_OK;

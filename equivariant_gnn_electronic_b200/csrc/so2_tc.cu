@@ -33,6 +33,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "so2_params.cuh"
 #include "so2_tc.cuh"
 #include "tc_ptx.cuh"
 
@@ -42,7 +43,8 @@ constexpr int kSA = 4;                 // A stages (128 x 64 bf16 = 16 KB each)
 constexpr int kSB = 2;                 // B stages (<= 512 x 64 bf16 = 64 KB each)
 constexpr int kAStage = 128 * 128;
 constexpr int kBStage = 512 * 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;   // 0 loader, 1 MMA, 2-9 producers, 10-13 epilogue
+constexpr int kProducers = 256;
 constexpr int kTmemCols = 512;
 
 struct SmemCtl {
@@ -51,8 +53,6 @@ struct SmemCtl {
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ float bf2f(uint16_t u) { return __uint_as_float(((uint32_t)u) << 16); }
 
 __device__ __forceinline__ void unpack8(const uint4& q, float* f) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -66,6 +66,63 @@ __device__ __forceinline__ void unpack8(const uint4& q, float* f) {
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// acc[i] (+)= sum_{mp < dl} co[mp] * z[mp*C + i], i < 32; loads are issued three
+// rows (12 x 16 B) at a time before their FMAs so that more of them are in flight.
+__device__ __forceinline__ void rot_acc1(float* acc, const __nv_bfloat16* z, int C, const float* co, int dl) {
+  for (int mp0 = 0; mp0 < dl; mp0 += 3) {
+    uint4 q[3][4];
+    float c[3];
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      const bool ok = mp0 + u < dl;
+      const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
+      c[u] = ok ? __ldg(co + mp0 + u) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 3; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float f[8];
+        unpack8(q[u][k], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[8 * k + i] += c[u] * f[i];
+      }
+  }
+}
+
+// Same for two coefficient rows at once (the +b and -b rows share z), two rows of z
+// (8 x 16 B) in flight per batch.
+__device__ __forceinline__ void rot_acc2(float* ap, float* am, const __nv_bfloat16* z, int C, const float* cop,
+                                         const float* com, int dl) {
+  for (int mp0 = 0; mp0 < dl; mp0 += 2) {
+    uint4 q[2][4];
+    float cp[2], cm[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const bool ok = mp0 + u < dl;
+      const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
+      cp[u] = ok ? __ldg(cop + mp0 + u) : 0.f;
+      cm[u] = ok ? __ldg(com + mp0 + u) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float f[8];
+        unpack8(q[u][k], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          ap[8 * k + i] += cp[u] * f[i];
+          am[8 * k + i] += cm[u] * f[i];
+        }
+      }
+  }
 }
 
 // Writes 32 values (columns [32*half, 32*half+32) of a 64-wide K chunk) of row r
@@ -98,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSA; ++i) {
-      tc::mbar_init(tc::smem_u32(&ctl->a_full[i]), 128);
+      tc::mbar_init(tc::smem_u32(&ctl->a_full[i]), kProducers);
       tc::mbar_init(tc::smem_u32(&ctl->a_empty[i]), 1);
     }
     for (int i = 0; i < kSB; ++i) {
@@ -185,9 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
       }
     }
     __syncwarp();
-  } else if (warp >= 2 && warp < 6) {
-    // ---------------- A producers: thread = tile row = edge ----------------
-    const int r = (warp - 2) * 32 + lane;
+  } else if (warp >= 2 && warp < 10) {
+    // ---------------- A producers: thread = (tile row = edge, 32-channel half) ----------------
+    const int pidx = (warp - 2) * 32 + lane;
+    const int r = pidx & 127;
+    const int half = pidx >> 7;
     const __nv_bfloat16* gsc = P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
     uint32_t ia = 0, it = 0;
     for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x, ++it) {
@@ -221,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
             int sa = ia % kSA;
             if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa]), ((ia / kSA) & 1) ^ 1, P.status, abort)) break;
             uint8_t* tile = Abuf + sa * kAStage;
-            for (int half = 0; half < 2; ++half) {
+            {
               float v[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = 0.f;
@@ -261,22 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
             const int cs = c2b * 64;
             const __nv_bfloat16* z = (cs < C) ? P.node_in + ((long long)s * P.L2 + l * l) * C + cs
                                               : P.node_in + ((long long)d * P.L2 + l * l) * C + (cs - C);
-            for (int half = 0; half < 2; ++half) {
+            {
               float acc[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) acc[i] = 0.f;
               if (valid) {
-                for (int mp = 0; mp < dl; ++mp) {
-                  const float co = Drow[mp];
-                  const uint4* zp = reinterpret_cast<const uint4*>(z + mp * C + half * 32);
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    float f[8];
-                    unpack8(__ldg(zp + q), f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[8 * q + i] += co * f[i];
-                  }
-                }
+                rot_acc1(acc, z + half * 32, C, Drow, dl);
                 const uint4* gp = reinterpret_cast<const uint4*>(gsc + l * C2 + cs + half * 32);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -308,25 +357,12 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
             const int cs = c2b * 64;
             const __nv_bfloat16* z = (cs < C) ? P.node_in + ((long long)s * P.L2 + l * l) * C + cs
                                               : P.node_in + ((long long)d * P.L2 + l * l) * C + (cs - C);
-            for (int half = 0; half < 2; ++half) {
+            {
               float ap[32], am[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) ap[i] = am[i] = 0.f;
               if (valid) {
-                for (int mp = 0; mp < dl; ++mp) {
-                  const float cp = Dp[mp], cm = Dm[mp];
-                  const uint4* zp = reinterpret_cast<const uint4*>(z + mp * C + half * 32);
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    float f[8];
-                    unpack8(__ldg(zp + q), f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                      ap[8 * q + i] += cp * f[i];
-                      am[8 * q + i] += cm * f[i];
-                    }
-                  }
-                }
+                rot_acc2(ap, am, z + half * 32, C, Dp, Dm, dl);
                 const uint4* gp = reinterpret_cast<const uint4*>(gsc + l * C2 + cs + half * 32);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -384,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
                                   pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
-            if (ps.block == 0) {
+            if (ps.block == 0 && P.with_logits) {
               for (int h = 0; h < H; ++h) {
                 const __nv_bfloat16* Ah = P.A + (long long)h * L * C + col;
                 float a = 0.f;
@@ -398,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
         tc::tc_fence_before();
         tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty));
         if (ps.kind == 0 && ps.last_of_kind) tc::mbar_arrive(tc::smem_u32(&ctl->gate_ready));
-        if (ps.kind == 1 && ps.block == 0 && ps.last_of_kind && valid) {
+        if (ps.kind == 1 && ps.block == 0 && ps.last_of_kind && valid && P.with_logits) {
           for (int h = 0; h < H; ++h) P.logits[e * H + h] = lg[h] + __bfloat162float(P.bA[h]);
         }
       }
@@ -459,14 +495,24 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
   reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-// Aggregation: one CTA per destination atom, thread = channel.
-template <int LM>
+// Aggregation: one CTA per destination atom, thread = channel.  Softmax statistics
+// per head first; then the incoming edges in batches of kAggB whose Wigner rows and
+// softmax weights are staged in shared memory; each thread issues all of an edge's
+// y loads before its FMAs.  Template parameters fix the kept rows (lmax, mmax).
+constexpr int kAggB = 8;
+constexpr int kAggWfl = 240;   // >= egnn_wigner_floats(6, 2) = 235
+
+template <int LM, int MM>
 __global__ void __launch_bounds__(128) agg_kernel(const __grid_constant__ TcParams P) {
   constexpr int L = LM + 1;
+  constexpr int NR = (MM == 0) ? L : (MM == 1 ? 3 * L - 2 : 5 * L - 6);   // kept rows
+  __shared__ float Ds[kAggB * kAggWfl];
+  __shared__ float ps[kAggB * 16];
+  __shared__ float hmx[16], hinv[16];
   const int d = blockIdx.x;
   const int c = threadIdx.x;
-  const int C = P.C, H = P.H;
-  const int h = c / (C / H);
+  const int C = P.C, H = P.H, hc = P.C / P.H;
+  const int h = c / hc;
   int e0 = P.row_ptr[d], e1 = P.row_ptr[d + 1];
   if (e0 < 0 || e1 < e0 || e1 > P.n_edges) {
     if (c == 0) egnn_flag(P.status, EGNN_DEV_BAD_GRAPH);
@@ -476,29 +522,52 @@ __global__ void __launch_bounds__(128) agg_kernel(const __grid_constant__ TcPara
   for (int e = e0; e < e1; ++e) mx = fmaxf(mx, P.logits[(long long)e * H + h]);
   float sum = 0.f;
   for (int e = e0; e < e1; ++e) sum += __expf(P.logits[(long long)e * H + h] - mx);
-  const float inv = e1 > e0 ? 1.0f / sum : 0.f;
+  if (c % hc == 0) {
+    hmx[h] = mx;
+    hinv[h] = e1 > e0 ? 1.0f / sum : 0.f;
+  }
+  // column of kept row (l, m) in y, and its Wigner offset, resolved at compile time
+  int col[NR], wo[NR], rl[NR];
+  {
+    int r = 0;
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+      const int ml = l < MM ? l : MM;
+#pragma unroll
+      for (int m = -ml; m <= ml; ++m) {
+        const int b = m < 0 ? -m : m;
+        col[r] = b == 0 ? l * C : P.ybase[b] + (m > 0 ? 0 : (L - b) * C) + (l - b) * C;
+        wo[r] = P.woff[l] + (m + ml) * (2 * l + 1);
+        rl[r] = l;
+        ++r;
+      }
+    }
+  }
   float acc[L * L];
 #pragma unroll
   for (int i = 0; i < L * L; ++i) acc[i] = 0.f;
-  const int mmax = P.mmax;
-  for (int e = e0; e < e1; ++e) {
-    const float pe = __expf(P.logits[(long long)e * H + h] - mx) * inv;
-    const __nv_bfloat16* y = P.Y + (long long)e * P.ncols_y;
-    const float* De = P.wig + (long long)e * P.wfl;
+  for (int eb = e0; eb < e1; eb += kAggB) {
+    const int nb = min(kAggB, e1 - eb);
+    __syncthreads();
+    for (int i = c; i < nb * P.wfl; i += 128) Ds[(i / P.wfl) * kAggWfl + i % P.wfl] = P.wig[(long long)eb * P.wfl + i];
+    for (int i = c; i < nb * H; i += 128) {
+      const int j = i / H, hh = i - j * H;
+      ps[j * 16 + hh] = __expf(P.logits[(long long)(eb + j) * H + hh] - hmx[hh]) * hinv[hh];
+    }
+    __syncthreads();
+    for (int j = 0; j < nb; ++j) {
+      const __nv_bfloat16* y = P.Y + (long long)(eb + j) * P.ncols_y + c;
+      float yv[NR];
 #pragma unroll
-    for (int l = 0; l < L; ++l) {
-      const int ml = l < mmax ? l : mmax;
-      const int dl = 2 * l + 1;
-      const float* Dl = De + P.woff[l];
-      for (int m = -ml; m <= ml; ++m) {
-        const int b = m < 0 ? -m : m;
-        int col;
-        if (b == 0) col = l * C;
-        else col = P.ybase[b] + (m > 0 ? 0 : (L - b) * C) + (l - b) * C;
-        const float yv = pe * __bfloat162float(y[col + c]);
-        const float* Dr = Dl + (m + ml) * dl;
+      for (int r = 0; r < NR; ++r) yv[r] = __bfloat162float(y[col[r]]);
+      const float pe = ps[j * 16 + h];
+      const float* Dj = Ds + j * kAggWfl;
 #pragma unroll
-        for (int mp = 0; mp < dl; ++mp) acc[l * l + mp] += Dr[mp] * yv;
+      for (int r = 0; r < NR; ++r) {
+        const int l = rl[r];
+        const float v = pe * yv[r];
+#pragma unroll
+        for (int mp = 0; mp < 2 * l + 1; ++mp) acc[l * l + mp] += Dj[wo[r] + mp] * v;
       }
     }
   }
@@ -510,11 +579,110 @@ __global__ void __launch_bounds__(128) agg_kernel(const __grid_constant__ TcPara
   }
 }
 
+template <int MM>
+cudaError_t launch_agg_mm(const TcParams& P, cudaStream_t st) {
+  switch (P.lmax) {
+    case 1: if (MM <= 1) agg_kernel<1, (MM <= 1 ? MM : 1)><<<P.n_atoms, 128, 0, st>>>(P); break;
+    case 2: agg_kernel<2, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
+    case 3: agg_kernel<3, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
+    case 4: agg_kernel<4, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
+    case 5: agg_kernel<5, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
+    default: agg_kernel<6, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
+  }
+  return cudaGetLastError();
+}
+
+// Hamiltonian head from y.  Persistent CTAs stage U^T (all L) in shared memory once,
+// then loop over groups of `te` edges: t = rotate-back of y, labels
+// h[L][M][k] = sum_c U^L[k][c] t[L, M, c] (lanes run over k: consecutive addresses in
+// U^T), block = sum of Clebsch-Gordan images.
+__global__ void __launch_bounds__(256) head_blocks_kernel(const __grid_constant__ TcParams P,
+                                                          const __grid_constant__ HeadTables Tb, HeadUPtrs Up,
+                                                          float* __restrict__ blocks, int te, int u_total) {
+  extern __shared__ float hsm[];
+  const int C = P.C, L = P.L, L2 = P.L2, mmax = P.mmax;
+  const int nlab = Tb.n_lab, norb = Tb.n_orb;
+  float* Us = hsm;                        // per L: [C][mult_L] at uoff(L) = C * sum_{L'<L} mult_L'
+  float* Ds = Us + u_total;               // [te][wfl]
+  float* Ts = Ds + te * P.wfl;            // [te][L2][C]
+  float* Ls = Ts + te * L2 * C;           // [te][nlab]
+  const int tid = threadIdx.x, nt = blockDim.x;
+  {
+    int uo = 0;
+    for (int Lq = 0; Lq <= P.lmax; ++Lq) {
+      const int mult = Tb.mult[Lq];
+      for (int i = tid; i < mult * C; i += nt) {
+        const int k = i / C, c = i - k * C;
+        Us[uo + c * mult + k] = __bfloat162float(Up.U[Lq][i]);
+      }
+      uo += mult * C;
+    }
+  }
+  const long long ngroups = (P.n_edges + te - 1) / te;
+  for (long long gi = blockIdx.x; gi < ngroups; gi += gridDim.x) {
+    const long long e0 = gi * te;
+    const int ne = (int)min((long long)te, P.n_edges - e0);
+    __syncthreads();
+    for (int i = tid; i < ne * P.wfl; i += nt) Ds[i] = P.wig[e0 * P.wfl + i];
+    __syncthreads();
+    for (int i = tid; i < ne * L2 * C; i += nt) {
+      const int e = i / (L2 * C), rr = i - e * L2 * C;
+      const int lm = rr / C, c = rr - lm * C;
+      int l = 0;
+      while ((l + 1) * (l + 1) <= lm) ++l;
+      const int mp = lm - l * l - l, ml = l < mmax ? l : mmax, dl = 2 * l + 1;
+      const float* Dl = Ds + e * P.wfl + P.woff[l];
+      const __nv_bfloat16* y = P.Y + (e0 + e) * (long long)P.ncols_y;
+      float v = 0.f;
+      for (int m = -ml; m <= ml; ++m) {
+        const int b = m < 0 ? -m : m;
+        const int col = b == 0 ? l * C : P.ybase[b] + (m > 0 ? 0 : (L - b) * C) + (l - b) * C;
+        v += Dl[(m + ml) * dl + (mp + l)] * __bfloat162float(y[col + c]);
+      }
+      Ts[i] = v;
+    }
+    __syncthreads();
+    for (int i = tid; i < ne * nlab; i += nt) {
+      const int e = i / nlab, q = i - e * nlab;
+      int Lq = 0;
+      while (Lq + 1 <= P.lmax && Tb.lab_off[Lq + 1] <= q) ++Lq;
+      const int mult = Tb.mult[Lq];
+      const int r = q - Tb.lab_off[Lq];
+      const int M = r / mult, k = r - M * mult;
+      int uo = 0;
+      for (int Lp = 0; Lp < Lq; ++Lp) uo += Tb.mult[Lp] * C;
+      const float* U = Us + uo + k;
+      const float* t = Ts + (e * L2 + Lq * Lq + M) * C;
+      float a = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < C; ++c) a += U[c * mult] * t[c];
+      Ls[i] = a;
+    }
+    __syncthreads();
+    for (int i = tid; i < ne * norb * norb; i += nt) {
+      const int e = i / (norb * norb), q = i - e * norb * norb;
+      const int ri = q / norb, cj = q - ri * norb;
+      const int a = Tb.orb_shell[ri], b = Tb.orb_shell[cj];
+      const int la = Tb.shell_l[a], lb = Tb.shell_l[b];
+      const int ia = ri - Tb.shell_off[a], jb = cj - Tb.shell_off[b];
+      float v = 0.f;
+      for (int Lc = (la > lb ? la - lb : lb - la); Lc <= la + lb; ++Lc) {
+        const int k = Tb.kidx[(a * Tb.n_shells + b) * 8 + Lc];
+        const float* cgm = Tb.cg + Tb.cg_off[(la * 4 + lb) * 8 + Lc] + (ia * (2 * lb + 1) + jb) * (2 * Lc + 1);
+        const float* h = Ls + e * nlab + Tb.lab_off[Lc] + k;
+        const int mult = Tb.mult[Lc];
+        for (int M = 0; M < 2 * Lc + 1; ++M) v += cgm[M] * h[M * mult];
+      }
+      blocks[(e0 + e) * norb * norb + q] = v;
+    }
+  }
+}
+
 }  // namespace
 
 size_t so2_tc_smem_bytes() { return kSA * kAStage + kSB * kBStage + sizeof(SmemCtl) + 1024; }
 
-cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st) {
+static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStream_t st) {
   long long total = P.wprep_bytes / 2;
   prep_weights_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(P, W.W2, W.W0, W.Wm[0][0], W.Wm[0][1],
                                                                       W.Wm[1][0], W.Wm[1][1], total,
@@ -529,14 +697,37 @@ cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  switch (P.lmax) {
-    case 0: agg_kernel<0><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 1: agg_kernel<1><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 2: agg_kernel<2><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 3: agg_kernel<3><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 4: agg_kernel<4><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 5: agg_kernel<5><<<P.n_atoms, 128, 0, st>>>(P); break;
-    default: agg_kernel<6><<<P.n_atoms, 128, 0, st>>>(P); break;
-  }
+  return cudaSuccess;
+}
+
+size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te) {
+  return sizeof(float) * (size_t)te * (P.wfl + P.L2 * P.C + n_lab);
+}
+
+cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
+                           float* blocks, cudaStream_t st) {
+  cudaError_t err = launch_tc_gemm(P, W, st);
+  if (err != cudaSuccess || P.n_edges == 0) return err;
+  int u_total = 0;
+  for (int Lq = 0; Lq <= P.lmax; ++Lq) u_total += T.mult[Lq] * P.C;
+  int te = 16;   // edges per group; aim at two CTAs per SM (<= 110 KB of shared memory each)
+  while (te > 1 && sizeof(float) * (size_t)u_total + head_tc_smem_bytes(P, T.n_lab, te) > 110 * 1024) te >>= 1;
+  size_t sm = sizeof(float) * (size_t)u_total + head_tc_smem_bytes(P, T.n_lab, te);
+  if (sm > 220 * 1024) return cudaErrorInvalidValue;
+  err = cudaFuncSetAttribute(head_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (err != cudaSuccess) return err;
+  long long groups = (P.n_edges + te - 1) / te;
+  int grid = (int)(groups < 4LL * P.grid ? groups : 4LL * P.grid);
+  head_blocks_kernel<<<grid, 256, sm, st>>>(P, T, U, blocks, te, u_total);
   return cudaGetLastError();
+}
+
+cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st) {
+  cudaError_t err = launch_tc_gemm(P, W, st);
+  if (err != cudaSuccess) return err;
+  switch (P.mmax) {
+    case 0: return launch_agg_mm<0>(P, st);
+    case 1: return launch_agg_mm<1>(P, st);
+    default: return launch_agg_mm<2>(P, st);
+  }
 }

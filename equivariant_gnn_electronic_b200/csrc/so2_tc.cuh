@@ -34,6 +34,7 @@ struct TcParams {
   __nv_bfloat16* Y;              // [n_edges][ncols_y]
   float* logits;                 // [n_edges][H]
   int32_t* status;
+  int with_logits;               // 1: layer (attention logits from SiLU(y0)); 0: head
   int npass;
   TcPass pass[16];
   int woff[8];
@@ -47,5 +48,13 @@ struct TcWeights {
 
 constexpr int kTcMaxGrid = 160;
 
+struct HeadTables;
+struct HeadUPtrs {
+  const __nv_bfloat16* U[8];
+};
+
 size_t so2_tc_smem_bytes();
 cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st);
+cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
+                           float* blocks, cudaStream_t st);
+size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te);

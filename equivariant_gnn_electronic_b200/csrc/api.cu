@@ -132,15 +132,17 @@ void tc_plan(const egnn_layer_desc* d, TcParams& P) {
     if (b > 0) P.pass[P.npass - 1].last_of_kind = 0;
   }
   P.ncols_y = ycol;
+  P.y0_bytes = L * C * 4;
+  P.y_row_bytes = P.y0_bytes + (ycol - L * C) * 2;
   P.gcols = L * 2 * C;
   P.wprep_bytes = boff;
 }
 
 struct TcWorkspace {
-  size_t wprep, gate, y, logits, total;
+  size_t wprep, gate, y, logits, node_h, af, total;
 };
 
-TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges) {
+TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_atoms) {
   TcParams P;
   memset(&P, 0, sizeof(P));
   tc_plan(d, P);
@@ -149,8 +151,11 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges) {
   w.wprep = 0;
   w.gate = align_up((size_t)P.wprep_bytes, 1024);
   w.y = w.gate + align_up((size_t)kTcMaxGrid * 128 * P.gcols * 2, 1024);
-  w.logits = w.y + align_up(E * P.ncols_y * 2, 1024);
-  w.total = w.logits + align_up(E * d->heads * 4, 1024) + 1024;
+  w.logits = w.y + align_up(E * (size_t)P.y_row_bytes, 1024);
+  w.node_h = w.logits + align_up(E * d->heads * 4, 1024);
+  size_t N = n_atoms > 0 ? (size_t)n_atoms : 0;
+  w.af = w.node_h + align_up(N * (d->lmax + 1) * (d->lmax + 1) * d->channels * 2, 1024);
+  w.total = w.af + align_up((size_t)d->heads * (d->lmax + 1) * d->channels * 4, 1024) + 1024;
   return w;
 }
 
@@ -158,7 +163,7 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges) {
 // workspace; returns false if the workspace is too small.
 bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_desc* desc, const So2Weights& W,
              const void* node_in, void* node_out, uint8_t* ws, int with_logits) {
-  TcWorkspace wl = tc_workspace(desc, g->n_edges);
+  TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
   memset(&T, 0, sizeof(T));
   tc_plan(desc, T);
   T.n_atoms = g->n_atoms;
@@ -192,9 +197,11 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   T.A = (const __nv_bfloat16*)W.A;
   T.bA = (const __nv_bfloat16*)W.bA;
   T.wprep = ws + wl.wprep;
-  T.gate_scratch = (__nv_bfloat16*)(ws + wl.gate);
-  T.Y = (__nv_bfloat16*)(ws + wl.y);
+  T.gate_scratch = (__half*)(ws + wl.gate);
+  T.Y = ws + wl.y;
   T.logits = (float*)(ws + wl.logits);
+  T.node_h = (__half*)(ws + wl.node_h);
+  T.Af = (float*)(ws + wl.af);
   TW.W2 = (const __nv_bfloat16*)W.W2;
   TW.W0 = (const __nv_bfloat16*)W.W0;
   for (int m = 0; m < 2; ++m)
@@ -294,11 +301,11 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
     case EGNN_WS_BUILD_GRAPH:
       return egnn_graph_workspace_bytes(n_atoms);
     case EGNN_WS_LAYER:
-      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc)) return tc_workspace(desc, n_edges).total;
+      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc)) return tc_workspace(desc, n_edges, n_atoms).total;
       return 256;
     case EGNN_WS_HAMILTONIAN:
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
-        return tc_workspace(desc, n_edges).total + 64 * 1024;
+        return tc_workspace(desc, n_edges, n_atoms).total + 64 * 1024;
       return 64 * 1024;
     default:
       return 0;
@@ -315,8 +322,9 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
   if (!weights || !node_in || !node_out || node_in == node_out) return EGNN_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)cuda_stream;
   if (tc_eligible(desc)) {
-    TcWorkspace wl = tc_workspace(desc, g->n_edges);
+    TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
     if (!workspace || ws_bytes < wl.total) return EGNN_ERR_INVALID_ARG;
+    if (((uintptr_t)weights | (uintptr_t)node_in | (uintptr_t)node_out) & 15) return EGNN_ERR_INVALID_ARG;
     uint8_t* ws = align1024(workspace);
     So2Weights W;
     carve_so2(W, (const char*)weights, desc, true);
@@ -391,7 +399,7 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
         real_cg(la, lb, Lc, cg);
       }
   const bool use_tc = tc_eligible(desc);
-  const size_t tc_bytes = use_tc ? tc_workspace(desc, g->n_edges).total : 0;
+  const size_t tc_bytes = use_tc ? tc_workspace(desc, g->n_edges, g->n_atoms).total : 0;
   size_t need = tc_bytes + kidx.size() * sizeof(int) + cg.size() * sizeof(float) + 64;
   if (ws_bytes < need) return EGNN_ERR_INVALID_ARG;
   uint8_t* ws_tc = align1024(workspace);
@@ -413,6 +421,7 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
   }
   if (use_tc) {
     if (g->n_edges == 0) return EGNN_OK;
+    if (((uintptr_t)head_weights | (uintptr_t)node_emb) & 15) return EGNN_ERR_INVALID_ARG;
     TcParams TP;
     TcWeights TW;
     fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, 0);

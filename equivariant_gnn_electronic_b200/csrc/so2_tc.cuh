@@ -1,6 +1,7 @@
 // Launch parameters of the tensor-core eSCN layer (CUDA path only).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,6 +21,8 @@ struct TcParams {
   long long n_edges;
   int n_tiles, grid;
   int lmax, mmax, C, H, K, L, L2, wfl, ncols_y, gcols;
+  int y_row_bytes;   // bytes of one edge's y record: y0 in fp32, then the |m| > 0 blocks in bf16
+  int y0_bytes;      // L * C * 4
   float rcut;
   const int32_t* row_ptr;
   const int32_t* src;
@@ -27,12 +30,14 @@ struct TcParams {
   const float* wig;
   const __nv_bfloat16* node_in;
   __nv_bfloat16* node_out;
+  __half* node_h;                // fp16 copy of node_in (exact), read by the A producers
   const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
   const uint8_t* wprep;
   long long wprep_bytes;
-  __nv_bfloat16* gate_scratch;   // [grid][128][gcols]
-  __nv_bfloat16* Y;              // [n_edges][ncols_y]
+  __half* gate_scratch;          // [grid][128][gcols] radial gates, fp16
+  uint8_t* Y;                    // [n_edges][y_row_bytes]
   float* logits;                 // [n_edges][H]
+  float* Af;                     // attention matrix A[H][L*C] in fp32 (workspace copy)
   int32_t* status;
   int with_logits;               // 1: layer (attention logits from SiLU(y0)); 0: head
   int npass;

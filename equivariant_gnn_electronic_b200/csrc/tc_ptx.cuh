@@ -46,11 +46,15 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // Bounded wait: gives up after ~2 s of wall time (or when *abort is set by another
 // role), records EGNN_DEV_WAIT_TIMEOUT and returns false.  Never traps.
+// `sleep_ns` > 0 makes a waiting warp yield its issue slot between polls (roles that
+// wait long and are not latency-critical), so it does not steal issue bandwidth from
+// the warps doing the work on the same SM sub-partition.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status,
-                                          volatile int* abort) {
+                                          volatile int* abort, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   while (true) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > 2000000000ull) {
@@ -90,7 +94,7 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulate.
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, 16-bit inputs (type in idesc), fp32 accumulate.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
@@ -138,6 +142,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 // Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M x N.
 __host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Instruction descriptor: f16 x f16 -> fp32, both K-major, M x N.
+__host__ __device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace tc

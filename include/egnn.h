@@ -155,6 +155,7 @@ egnn_status egnn_build_graph_noalloc(const double* pos, const int32_t* species, 
  *   is l*C + c, of y+-m is (l-m)*C + c; gate index l*2C + c2.
  * node_in / node_out  device [n_atoms][(lmax+1)^2][C], fp32 or bf16 per dtype;
  *   must not overlap.  An atom without incoming edges gets out = in.
+ *   weights, node_in and node_out must be 16-byte aligned (EGNN_ERR_INVALID_ARG).
  * g must come from egnn_build_graph with the same lmax/mmax and rcut.
  */
 egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_desc* desc,

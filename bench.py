@@ -46,6 +46,25 @@ def layer_flops_per_edge(w) -> float:
     return 2.0 * macs
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_traffic_hfo2_3000.json")
+
+
+def measured_layer_traffic(n_edges: int):
+    """DRAM bytes of one layer call from the committed ncu capture, scaled to n_edges by the
+    edge count (the traffic grows with the edges), or None if the kernel sources changed
+    since the counters were taken."""
+    import hashlib
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    d = json.load(open(TRAFFIC_FILE))
+    h = hashlib.sha1()
+    for f in d["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != d["sources_sha1"]:
+        return None, "kernel sources changed since the capture"
+    return d["bytes_per_edge"] * n_edges, f"scaled from {d['workload']} ({d['edges']} edges) by edge count"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -273,8 +292,10 @@ def main():
     flops = layer_flops_per_edge(w) * E
     achieved = flops / layer_avg_s / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    roofline = {"bound": "tensor", "kernel": "egnn_layer_forward", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+    traffic, traffic_note = measured_layer_traffic(E)
+    roofline = {"bound": "tensor", "kernel": "egnn_layer_forward (prep, to_f16, so2_tc, logits, agg)",
+                "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "traffic_note": traffic_note,
                 "peak_source": f"bf16_tflops_sustained ({peak_src})",
                 "flops_per_launch": flops, "layer_ms": 1e3 * layer_avg_s,
                 "layer_edges_per_s": E / layer_avg_s}

@@ -116,6 +116,7 @@ void tc_plan(const egnn_layer_desc* d, TcParams& P) {
       q.n_off = off;
       q.nk = nk;
       q.last_of_kind = 0;
+      q.np = 0;
       q.boff = boff;
       boff += (long long)q.n * nk * 128;
     }
@@ -123,13 +124,27 @@ void tc_plan(const egnn_layer_desc* d, TcParams& P) {
   };
   add(0, 0, L * 2 * C, C / 64);
   int ycol = 0;
-  for (int b = 0; b <= d->mmax; ++b) {
-    int nb = b == 0 ? L * C : 2 * (L - b) * C;
-    int kb = b == 0 ? L * 2 * C : 2 * (L - b) * 2 * C;
+  P.ybase[0] = ycol;
+  add(1, 0, L * C, L * 2 * C / 64);
+  ycol += L * C;
+  for (int b = 1; b <= d->mmax; ++b) {
+    // rows [o0, o0 + np) of y+ and of y-: B = [W_b1 rows ; W_b2 rows] for those outputs,
+    // K = the (l, channel) index shared by x+ and x- (each K block feeds 4 MMAs)
+    const int nC = (L - b) * C, kblocks = (L - b) * 2 * C / 64;
     P.ybase[b] = ycol;
-    ycol += nb;
-    add(1, b, nb, kb / 64);
-    if (b > 0) P.pass[P.npass - 1].last_of_kind = 0;
+    ycol += 2 * nC;
+    for (int o0 = 0; o0 < nC; o0 += 256) {
+      TcPass& q = P.pass[P.npass++];
+      q.kind = 1;
+      q.block = b;
+      q.np = nC - o0 < 256 ? nC - o0 : 256;
+      q.n = 2 * q.np;
+      q.n_off = o0;
+      q.nk = kblocks;
+      q.last_of_kind = 0;
+      q.boff = boff;
+      boff += (long long)q.n * kblocks * 128;
+    }
   }
   P.ncols_y = ycol;
   P.y0_bytes = L * C * 4;

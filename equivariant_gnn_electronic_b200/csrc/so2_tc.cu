@@ -25,7 +25,8 @@
 //                                form [[W_b1, -W_b2], [W_b2, W_b1]] (b > 0)
 //                                -> y_e (bf16).
 //                 Warp roles: 0 bulk-copies B tiles, 1 issues MMAs (one thread)
-//                 and owns TMEM, 2-5 build A tiles, 6-9 drain TMEM.
+//                 and owns TMEM, 2-9 build A tiles (8 lanes per 128-byte row slice so
+//                 that gathers are coalesced), 10-13 drain TMEM.
 //   agg           one CTA per destination atom, thread = channel pair: attention
 //                 logits from SiLU(y0), online softmax over the atom's incoming
 //                 edges, rotate y back with the kept rows of D^l(R_e), weighted
@@ -43,8 +44,9 @@ constexpr int kSA = 4;                 // A stages (128 x 64 bf16 = 16 KB each)
 constexpr int kSB = 2;                 // B stages (<= 512 x 64 bf16 = 64 KB each)
 constexpr int kAStage = 128 * 128;
 constexpr int kBStage = 512 * 128;
-constexpr int kThreads = 448;   // 0 loader, 1 MMA, 2-9 producers, 10-13 epilogue
-constexpr int kProducers = 256;
+constexpr int kPW = 8;                         // producer warps (256 threads: 8 lanes per row, 32 rows per step)
+constexpr int kProducers = kPW * 32;
+constexpr int kThreads = (2 + kPW + 4) * 32;   // 0 loader, 1 MMA, producers, 4 epilogue warps
 constexpr int kTmemCols = 512;
 
 constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = 128: 2 chunks
@@ -70,25 +72,27 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// acc[i] (+)= sum_{mp < dl} co[mp] * z[mp*C + 2i .. 2i+1] for 32 fp16 channels held as
-// 16 half2, in packed fp16 arithmetic (one HFMA2 per channel pair and row); three rows
-// of z (12 x 16 B) are loaded before their FMAs.
+// Producer helpers.  A thread owns NCH consecutive fp16 channels (NCH / 2 half2) of one
+// tile row.  acc (+)= sum_{mp < dl} co[mp] * z[mp * C + channels] in packed fp16
+// (one HFMA2 per channel pair and row); BATCH rows of z are loaded before their FMAs.
+template <int NCH, int BATCH>
 __device__ __forceinline__ void rot_h1(__half2* acc, const __half* z, int C, const float* co, int dl) {
-  for (int mp0 = 0; mp0 < dl; mp0 += 3) {
-    uint4 q[3][4];
-    __half2 c[3];
+  constexpr int Q = NCH / 8;                 // 16-byte loads per row
+  for (int mp0 = 0; mp0 < dl; mp0 += BATCH) {
+    uint4 q[BATCH][Q];
+    __half2 c[BATCH];
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
+    for (int u = 0; u < BATCH; ++u) {
       const bool ok = mp0 + u < dl;
       const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
+      for (int k = 0; k < Q; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
       c[u] = __float2half2_rn(ok ? __ldg(co + mp0 + u) : 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < 3; ++u)
+    for (int u = 0; u < BATCH; ++u)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < Q; ++k) {
         const __half2* h = reinterpret_cast<const __half2*>(&q[u][k]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[4 * k + i] = __hfma2(c[u], h[i], acc[4 * k + i]);
@@ -96,26 +100,27 @@ __device__ __forceinline__ void rot_h1(__half2* acc, const __half* z, int C, con
   }
 }
 
-// Same for two coefficient rows at once (the +b and -b rows share z), two rows of z
-// (8 x 16 B) in flight per batch.
+// Same for the two coefficient rows of the (+b, -b) pair, which share z.
+template <int NCH, int BATCH>
 __device__ __forceinline__ void rot_h2(__half2* ap, __half2* am, const __half* z, int C, const float* cop,
                                        const float* com, int dl) {
-  for (int mp0 = 0; mp0 < dl; mp0 += 2) {
-    uint4 q[2][4];
-    __half2 cp[2], cm[2];
+  constexpr int Q = NCH / 8;
+  for (int mp0 = 0; mp0 < dl; mp0 += BATCH) {
+    uint4 q[BATCH][Q];
+    __half2 cp[BATCH], cm[BATCH];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < BATCH; ++u) {
       const bool ok = mp0 + u < dl;
       const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
+      for (int k = 0; k < Q; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
       cp[u] = __float2half2_rn(ok ? __ldg(cop + mp0 + u) : 0.f);
       cm[u] = __float2half2_rn(ok ? __ldg(com + mp0 + u) : 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int u = 0; u < BATCH; ++u)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < Q; ++k) {
         const __half2* h = reinterpret_cast<const __half2*>(&q[u][k]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -126,11 +131,12 @@ __device__ __forceinline__ void rot_h2(__half2* ap, __half2* am, const __half* z
   }
 }
 
-// acc[i] *= g[i] for 32 fp16 channels (16 half2) read from the gate scratch.
+// acc *= g for the thread's NCH fp16 channels read from the gate scratch.
+template <int NCH>
 __device__ __forceinline__ void gate_mul(__half2* acc, const __half* g) {
   const uint4* gp = reinterpret_cast<const uint4*>(g);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < NCH / 8; ++k) {
     const uint4 w = gp[k];
     const __half2* h = reinterpret_cast<const __half2*>(&w);
 #pragma unroll
@@ -138,12 +144,13 @@ __device__ __forceinline__ void gate_mul(__half2* acc, const __half* g) {
   }
 }
 
-// Writes 32 fp16 values (16 half2) as columns [32*half, 32*half+32) of row r of a
-// 128B-swizzled K-major tile.
-__device__ __forceinline__ void store_row_h(uint8_t* tile, int r, int half, const __half2* v) {
+// Writes NCH fp16 values (NCH / 2 half2) as columns [NCH*part, NCH*part + NCH) of row r of a
+// 128B-swizzled K-major tile (16-byte chunk c of row r sits at position c ^ (r & 7)).
+template <int NCH>
+__device__ __forceinline__ void store_row_h(uint8_t* tile, int r, int part, const __half2* v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int chunk = half * 4 + q;
+  for (int q = 0; q < NCH / 8; ++q) {
+    const int chunk = part * (NCH / 8) + q;
     uint4 w;
     w.x = *reinterpret_cast<const uint32_t*>(&v[4 * q + 0]);
     w.y = *reinterpret_cast<const uint32_t*>(&v[4 * q + 1]);
@@ -158,18 +165,94 @@ __device__ __forceinline__ uint32_t pack2h(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Writes 32 fp32 values, rounded to fp16, as columns [32*half, 32*half+32) of row r
+// Writes NCH fp32 values, rounded to fp16, as columns [NCH*part, NCH*part + NCH) of row r
 // of a 128B-swizzled K-major tile.
-__device__ __forceinline__ void store_row32(uint8_t* tile, int r, int half, const float* v) {
+template <int NCH>
+__device__ __forceinline__ void store_row_f(uint8_t* tile, int r, int part, const float* v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    int chunk = half * 4 + q;
+  for (int q = 0; q < NCH / 8; ++q) {
+    const int chunk = part * (NCH / 8) + q;
     uint4 w;
     w.x = pack2h(v[8 * q + 0], v[8 * q + 1]);
     w.y = pack2h(v[8 * q + 2], v[8 * q + 3]);
     w.z = pack2h(v[8 * q + 4], v[8 * q + 5]);
     w.w = pack2h(v[8 * q + 6], v[8 * q + 7]);
     *reinterpret_cast<uint4*>(tile + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
+  }
+}
+
+// Epilogue store of one 32-column group of a pass (thread = edge row): gate passes
+// add b2 and keep fp16 gates in the CTA's scratch; SO(2) passes write y (y0 in fp32,
+// the |m| > 0 blocks in bf16).
+__device__ __forceinline__ void epi_store(const TcParams& P, const TcPass& ps, __half* gsc, long long e, bool valid,
+                                          int g, const uint32_t* ru) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ru[i]);
+  int col = ps.n_off + g;
+  if (ps.kind == 1 && ps.block > 0 && g >= ps.np) col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
+  if (ps.kind == 0) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += __bfloat162float(P.b2[col + i]);
+    uint4* dst = reinterpret_cast<uint4*>(gsc + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pack2h(v[8 * q], v[8 * q + 1]), pack2h(v[8 * q + 2], v[8 * q + 3]),
+                          pack2h(v[8 * q + 4], v[8 * q + 5]), pack2h(v[8 * q + 6], v[8 * q + 7]));
+  } else if (valid) {
+    uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
+    if (ps.block == 0) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = make_uint4(ru[4 * q], ru[4 * q + 1], ru[4 * q + 2], ru[4 * q + 3]);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) +
+                                            (P.ybase[ps.block] - P.ybase[1]) + col);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
+                            pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
+    }
+  }
+}
+
+// Attention logits a_{e,h} = A[h] . SiLU(y0_e) + bA[h], one warp per edge: lanes
+// read y0 (fp32, coalesced) and the fp32 copy of A staged in shared memory, then the
+// heads' partial sums are reduced across the warp.
+__global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ float As[];                 // [H][L*C]
+  const int LC = P.L * P.C, H = P.H;
+  for (int i = threadIdx.x; i < H * LC; i += blockDim.x) As[i] = P.Af[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < P.n_edges; e += nw) {
+    const float* y0 = reinterpret_cast<const float*>(P.Y + e * (long long)P.y_row_bytes);
+    float a[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) a[h] = 0.f;
+    float yv[28];                                // LC <= 7 * 128 = 896 = 28 * 32: all loads first
+#pragma unroll
+    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 28; ++k) {
+      const int j = lane + 32 * k;
+      if (j < LC) {
+        const float sv = yv[k] / (1.0f + __expf(-yv[k]));
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+          if (h < H) a[h] += As[h * LC + j] * sv;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+      if (h < H) {
+        float x = a[h];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (lane == 0) P.logits[e * H + h] = x + __bfloat162float(P.bA[h]);
+      }
+    }
   }
 }
 
@@ -257,33 +340,61 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
             hid_waited = true;
           }
           tc::tc_fence_after();
-          for (int j = 0; j < ps.nk; ++j, ++ib) {
-            const int sb = ib % kSB;
-            int sa = 0;
-            uint32_t a_base;
-            if (ps.kind == 0) {
-              a_base = H_u32 + j * kAStage;           // hidden layer, resident for the whole tile
-            } else {
-              sa = ia % kSA;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sa]), (ia / kSA) & 1, P.status, abort, 32)) break;
-              a_base = A_u32 + sa * kAStage;
-            }
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort, 32)) break;
-            tc::tc_fence_after();
+          if (ps.kind == 1 && ps.block > 0) {
+            // y+ += x+ W1^T - x- W2^T ; y- += x+ W2^T + x- W1^T, one K block of 64 per step
+            const int np = ps.np;
+            for (int kb = 0; kb < ps.nk; ++kb, ++ib, ia += 2) {
+              const int sb = ib % kSB, sp = ia % kSA, sm = (ia + 1) % kSA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sp]), (ia / kSA) & 1, P.status, abort, 32)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sm]), ((ia + 1) / kSA) & 1, P.status, abort, 32)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort, 32)) break;
+              tc::tc_fence_after();
+              const uint32_t idn = tc::idesc_f16(128, np), idneg = tc::idesc_f16(128, np, true);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              uint64_t ad = tc::sw128_desc(a_base + ks * 32);
-              for (int n0 = 0; n0 < ps.n; n0 += 256) {
-                int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
-                uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + n0 * 128 + ks * 32);
-                tc::mma_bf16(tmem + n0, ad, bd, tc::idesc_f16(128, ns), (j > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ap = tc::sw128_desc(A_u32 + sp * kAStage + ks * 32);
+                const uint64_t am = tc::sw128_desc(A_u32 + sm * kAStage + ks * 32);
+                const uint64_t b1 = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
+                const uint64_t b2 = tc::sw128_desc(B_u32 + sb * kBStage + np * 128 + ks * 32);
+                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                tc::mma_bf16(tmem, ap, b1, idn, acc);
+                tc::mma_bf16(tmem, am, b2, idneg, 1u);
+                tc::mma_bf16(tmem + np, ap, b2, idn, acc);
+                tc::mma_bf16(tmem + np, am, b1, idn, 1u);
               }
+              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sp]));
+              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sm]));
+              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
             }
-            if (ps.kind != 0) {
-              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
-              ++ia;
+          } else {
+            for (int j = 0; j < ps.nk; ++j, ++ib) {
+              const int sb = ib % kSB;
+              int sa = 0;
+              uint32_t a_base;
+              if (ps.kind == 0) {
+                a_base = H_u32 + j * kAStage;           // hidden layer, resident for the whole tile
+              } else {
+                sa = ia % kSA;
+                if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sa]), (ia / kSA) & 1, P.status, abort, 32)) break;
+                a_base = A_u32 + sa * kAStage;
+              }
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort, 32)) break;
+              tc::tc_fence_after();
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                uint64_t ad = tc::sw128_desc(a_base + ks * 32);
+                for (int n0 = 0; n0 < ps.n; n0 += 256) {
+                  int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
+                  uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + n0 * 128 + ks * 32);
+                  tc::mma_bf16(tmem + n0, ad, bd, tc::idesc_f16(128, ns), (j > 0 || ks > 0) ? 1u : 0u);
+                }
+              }
+              if (ps.kind != 0) {
+                tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
+                ++ia;
+              }
+              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
             }
-            tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
           }
           if (ps.kind == 0 && ps.last_of_kind) tc::mma_commit(tc::smem_u32(&ctl->hid_empty));
           tc::mma_commit(tc::smem_u32(&ctl->acc_full));
@@ -296,68 +407,78 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
       }
     }
     __syncwarp();
-  } else if (warp >= 2 && warp < 10) {
-    // ---------------- A producers: thread = (tile row = edge, 32-channel half) ----------------
+  } else if (warp >= 2 && warp < 2 + kPW) {
+    // ---------------- A producers ----------------
+    // Coalesced mapping: the 8 lanes of a group own the eight 16-byte chunks (8 fp16
+    // channels each) of one 128-byte row slice, a warp covers 4 rows per step, and each
+    // thread walks 4 rows (rb, rb+32, rb+64, rb+96).  Every warp-wide load then touches
+    // 4 cache lines instead of 32, and a row's Wigner coefficients are broadcasts.
     const int pidx = (warp - 2) * 32 + lane;
-    const int r = pidx & 127;
-    const int half = pidx >> 7;
-    const __half* gsc = P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
+    const int q = pidx & 7;                    // 16-byte chunk within a 64-channel slice
+    const int rb = pidx >> 3;                  // 0..31
     uint32_t ia = 0, it = 0;
     for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x, ++it) {
-      const long long e = (long long)t * 128 + r;
-      const bool valid = e < E;
-      int s = 0, d = 0;
-      float dist = 0.f;
-      if (valid) {
-        s = P.src[e];
-        int lo = 0, hi = P.n_atoms;
-        while (hi - lo > 1) {
-          int mid = (lo + hi) >> 1;
-          if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+      int srcs[4], dsts[4];
+      float dists[4];
+      bool valids[4];
+      const float* Dr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const long long e = (long long)t * 128 + rb + 32 * u;
+        valids[u] = e < E;
+        int sv = 0, dv = 0;
+        float di = 0.f;
+        if (valids[u]) {
+          sv = P.src[e];
+          int lo = 0, hi = P.n_atoms;
+          while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+          }
+          dv = lo;
+          if (sv < 0 || sv >= P.n_atoms) {
+            egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
+            sv = dv;
+          }
+          di = P.dist[e];
         }
-        d = lo;
-        if (s < 0 || s >= P.n_atoms) {
-          egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
-          s = d;
-        }
-        dist = P.dist[e];
+        srcs[u] = sv;
+        dsts[u] = dv;
+        dists[u] = di;
+        Dr[u] = P.wig + (valids[u] ? e : 0) * (long long)P.wfl;
       }
-      const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl;
       // radial hidden layer SiLU(W1 rho(|r_e|) + b1), once per tile, into Hbuf
       if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty), (it & 1) ^ 1, P.status, abort, 64)) break;
       {
         const float mu_step = P.rcut / (float)(K - 1);
         const float inv2s2 = 1.0f / (2.0f * mu_step * mu_step);
-        for (int j = 0; j < C / 64; ++j) {
-          float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          if (valid) {
-            const int c0 = j * 64 + half * 32;
+        for (int u = 0; u < 4; ++u) {
+          const int r = rb + 32 * u;
+          for (int j = 0; j < C / 64; ++j) {
+            const int c0 = j * 64 + q * 8;
+            float v[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(P.b1[c0 + i]);
-            for (int k0 = 0; k0 < K; k0 += 8) {
-              float rho[8];
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
+            if (valids[u]) {
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const float dd = dist - (k0 + u) * mu_step;
-                rho[u] = (k0 + u < K) ? __expf(-dd * dd * inv2s2) : 0.f;
+              for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(P.b1[c0 + i]);
+              for (int k = 0; k < K; ++k) {
+                const float dd = dists[u] - k * mu_step;
+                const float rho = __expf(-dd * dd * inv2s2);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] += __bfloat162float(P.W1[(c0 + i) * K + k]) * rho;
               }
-#pragma unroll 4
-              for (int i = 0; i < 32; ++i) {
-                // W1 row (c0 + i), columns k0..k0+7 (K is a multiple of 8 or padded by the bound)
-                const __nv_bfloat16* wr = P.W1 + (c0 + i) * K + k0;
-                float a = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                  if (k0 + u < K) a += __bfloat162float(wr[u]) * rho[u];
-                v[i] += a;
-              }
+              for (int i = 0; i < 8; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
+            uint4 w;
+            w.x = pack2h(v[0], v[1]);
+            w.y = pack2h(v[2], v[3]);
+            w.z = pack2h(v[4], v[5]);
+            w.w = pack2h(v[6], v[7]);
+            *reinterpret_cast<uint4*>(Hbuf + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
           }
-          store_row32(Hbuf + j * kAStage, r, half, v);
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(tc::smem_u32(&ctl->hid_full));
@@ -371,63 +492,73 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
           gate_waited = true;
         }
         const int b = ps.block;
-        if (b == 0) {
-          for (int j = 0; j < ps.nk; ++j, ++ia) {
-            int sa = ia % kSA;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa]), ((ia / kSA) & 1) ^ 1, P.status, abort, 32)) break;
-            uint8_t* tile = Abuf + sa * kAStage;
-            const int l = j / (C2 / 64), c2b = j % (C2 / 64);
-            const int dl = 2 * l + 1, ml = l < P.mmax ? l : P.mmax;
-            const float* Drow = De + P.woff[l] + ml * dl;          // row m = 0
-            const int cs = c2b * 64;
-            const __half* z = (cs < C) ? P.node_h + ((long long)s * P.L2 + l * l) * C + cs
-                                       : P.node_h + ((long long)d * P.L2 + l * l) * C + (cs - C);
-            {
-              __half2 acc[16];
+        const bool pair = b > 0;
+        const int nchunk = pair ? ps.nk : ps.nk;   // K blocks (pairs) or chunks
+        for (int j = 0; j < nchunk; ++j) {
+          const int sa0 = ia % kSA, sa1 = (ia + 1) % kSA;
+          if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa0]), ((ia / kSA) & 1) ^ 1, P.status, abort, 32)) break;
+          if (pair &&
+              !tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa1]), (((ia + 1) / kSA) & 1) ^ 1, P.status, abort, 32))
+            break;
+          const int l = b + j / (C2 / 64), c2b = j % (C2 / 64);
+          const int dl = 2 * l + 1, ml = l < P.mmax ? l : P.mmax;
+          const int rp = ml + b, rm = ml - b;      // kept rows m = +b and m = -b (b = 0: the same)
+          const int cs = c2b * 64;
+          const int coff = (cs < C ? cs : cs - C) + q * 8;
+          __half2 ap[4][4], am[4][4];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) acc[i] = __float2half2_rn(0.f);
-              if (valid) {
-                rot_h1(acc, z + half * 32, C, Drow, dl);
-                gate_mul(acc, gsc + l * C2 + cs + half * 32);
-              }
-              store_row_h(tile, r, half, acc);
-            }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa]));
-          }
-        } else {
-          // chunk pairs (+b, -b) of the same (l, 64 channels): z is read once for both
-          for (int j = 0; j < ps.nk; j += 2, ia += 2) {
-            int sa0 = ia % kSA, sa1 = (ia + 1) % kSA;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa0]), ((ia / kSA) & 1) ^ 1, P.status, abort, 32)) break;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa1]), (((ia + 1) / kSA) & 1) ^ 1, P.status, abort, 32))
-              break;
-            uint8_t* tp = Abuf + sa0 * kAStage;
-            uint8_t* tm = Abuf + sa1 * kAStage;
-            const int q2 = j >> 1;
-            const int l = b + q2 / (C2 / 64), c2b = q2 % (C2 / 64);
-            const int dl = 2 * l + 1, ml = l < P.mmax ? l : P.mmax;
-            const float* Dp = De + P.woff[l] + (ml + b) * dl;
-            const float* Dm = De + P.woff[l] + (ml - b) * dl;
-            const int cs = c2b * 64;
-            const __half* z = (cs < C) ? P.node_h + ((long long)s * P.L2 + l * l) * C + cs
-                                       : P.node_h + ((long long)d * P.L2 + l * l) * C + (cs - C);
-            {
-              __half2 ap[16], am[16];
+          for (int u = 0; u < 4; ++u)
 #pragma unroll
-              for (int i = 0; i < 16; ++i) ap[i] = am[i] = __float2half2_rn(0.f);
-              if (valid) {
-                rot_h2(ap, am, z + half * 32, C, Dp, Dm, dl);
-                gate_mul(ap, gsc + l * C2 + cs + half * 32);
-                gate_mul(am, gsc + l * C2 + cs + half * 32);
-              }
-              store_row_h(tp, r, half, ap);
-              store_row_h(tm, r, half, am);
+            for (int i = 0; i < 4; ++i) ap[u][i] = am[u][i] = __float2half2_rn(0.f);
+          for (int mp = 0; mp < dl; ++mp) {
+            uint4 zq[4];
+            __half2 cp[4], cm[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int node = cs < C ? srcs[u] : dsts[u];
+              zq[u] = valids[u] ? __ldg(reinterpret_cast<const uint4*>(
+                                      P.node_h + ((long long)node * P.L2 + l * l + mp) * C + coff))
+                                : make_uint4(0, 0, 0, 0);
+              const float* Dl = Dr[u] + P.woff[l];
+              cp[u] = __float2half2_rn(valids[u] ? __ldg(Dl + rp * dl + mp) : 0.f);
+              cm[u] = __float2half2_rn(valids[u] && pair ? __ldg(Dl + rm * dl + mp) : 0.f);
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa0]));
-            tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa1]));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __half2* h = reinterpret_cast<const __half2*>(&zq[u]);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                ap[u][i] = __hfma2(cp[u], h[i], ap[u][i]);
+                if (pair) am[u][i] = __hfma2(cm[u], h[i], am[u][i]);
+              }
+            }
           }
+          uint8_t* tp = Abuf + sa0 * kAStage;
+          uint8_t* tm = Abuf + sa1 * kAStage;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = rb + 32 * u;
+            const uint4 gw = *reinterpret_cast<const uint4*>(P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols +
+                                                             l * C2 + cs + q * 8);
+            const __half2* g = reinterpret_cast<const __half2*>(&gw);
+            uint4 wp, wm;
+            uint32_t* pp = reinterpret_cast<uint32_t*>(&wp);
+            uint32_t* pm = reinterpret_cast<uint32_t*>(&wm);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __half2 xp = __hmul2(ap[u][i], g[i]);
+              const __half2 xm = __hmul2(am[u][i], g[i]);
+              pp[i] = *reinterpret_cast<const uint32_t*>(&xp);
+              pm[i] = *reinterpret_cast<const uint32_t*>(&xm);
+            }
+            const int off = r * 128 + ((q ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(tp + off) = wp;
+            if (pair) *reinterpret_cast<uint4*>(tm + off) = wm;
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa0]));
+          if (pair) tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa1]));
+          ia += pair ? 2 : 1;
         }
       }
     }
@@ -438,72 +569,23 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
     __half* gsc = P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
     uint32_t ip = 0;
-    const int H = P.H;
     for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x) {
       const long long e = (long long)t * 128 + r;
       const bool valid = e < E;
-      float lg[16];
-#pragma unroll
-      for (int h = 0; h < 16; ++h) lg[h] = 0.f;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
         if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full), ip & 1, P.status, abort, 256)) break;
         tc::tc_fence_after();
         for (int g = 0; g < ps.n; g += 32) {
-          float v[32];
-          tc::tmem_ld32(tl + g, v);
-          const int col = ps.n_off + g;
-          if (ps.kind == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] += __bfloat162float(P.b2[col + i]);
-            uint4* dst = reinterpret_cast<uint4*>(gsc + col);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack2h(v[8 * q], v[8 * q + 1]), pack2h(v[8 * q + 2], v[8 * q + 3]),
-                                  pack2h(v[8 * q + 4], v[8 * q + 5]), pack2h(v[8 * q + 6], v[8 * q + 7]));
-          } else if (valid) {
-            uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
-            if (ps.block == 0) {               // y0 stays fp32
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + col);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                    __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
-              if (P.with_logits) {             // a_h += A[h, col..col+31] . SiLU(y0[col..col+31])
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                  if (h < H) {
-                    const float4* Ah = reinterpret_cast<const float4*>(P.Af + (long long)h * P.L * P.C + col);
-                    float a = 0.f;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                      const float4 w4 = __ldg(Ah + q);
-                      a += w4.x * v[4 * q] + w4.y * v[4 * q + 1] + w4.z * v[4 * q + 2] + w4.w * v[4 * q + 3];
-                    }
-                    lg[h] += a;
-                  }
-                }
-              }
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) +
-                                                    (P.ybase[ps.block] - P.ybase[1]) + col);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
-                                    pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
-            }
-          }
+          uint32_t ra[32];
+          tc::tmem_ld32_issue(tl + g, ra);
+          tc::tmem_ld_wait(ra);
+          epi_store(P, ps, gsc, e, valid, g, ra);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty));
         if (ps.kind == 0 && ps.last_of_kind) tc::mbar_arrive(tc::smem_u32(&ctl->gate_ready));
-        if (ps.kind == 1 && ps.block == 0 && ps.last_of_kind && valid && P.with_logits) {
-#pragma unroll
-          for (int h = 0; h < 16; ++h)
-            if (h < H) P.logits[e * H + h] = lg[h] + __bfloat162float(P.bA[h]);
-        }
+
       }
     }
   }
@@ -538,26 +620,19 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
   int chunk_pos = pos >> 4;
   int chunk = chunk_pos ^ (r & 7);
   int k = chunk * 8 + ((pos & 15) >> 1);
-  int row = ps.n_off + r;   // output row of the block matrix
+  const int row = ps.n_off + r;   // output row (gate and m = 0 passes)
   float v = 0.f;
   if (ps.kind == 0) {
     v = __bfloat162float(W2[(long long)row * C + j * 64 + k]);
   } else if (ps.block == 0) {
     v = __bfloat162float(W0[(long long)row * (L * C2) + j * 64 + k]);
   } else {
+    // rows [0, np) = W_b1[n_off + r], rows [np, 2np) = W_b2[n_off + r - np]; K block j is
+    // the shared (l - b, channel) index of x+ and x-
     const int b = ps.block, nb = L - b;
-    const __nv_bfloat16* Wa = b == 1 ? Wm1a : Wm2a;
-    const __nv_bfloat16* Wb = b == 1 ? Wm1b : Wm2b;
-    const int q2 = j >> 1, sgn = j & 1;
-    const int lq = q2 / (C2 / 64), c2b = q2 % (C2 / 64);
-    const int kg = lq * C2 + c2b * 64 + k;        // index inside x+ or x-
-    const int ld = nb * C2;
-    if (row < nb * C) {                                // y+ = W_b1 x+ - W_b2 x-
-      v = sgn == 0 ? __bfloat162float(Wa[(long long)row * ld + kg]) : -__bfloat162float(Wb[(long long)row * ld + kg]);
-    } else {                                           // y- = W_b2 x+ + W_b1 x-
-      int o = row - nb * C;
-      v = sgn == 0 ? __bfloat162float(Wb[(long long)o * ld + kg]) : __bfloat162float(Wa[(long long)o * ld + kg]);
-    }
+    const __nv_bfloat16* W = (b == 1 ? (r < ps.np ? Wm1a : Wm1b) : (r < ps.np ? Wm2a : Wm2b));
+    const int o = ps.n_off + (r < ps.np ? r : r - ps.np);
+    v = __bfloat162float(W[(long long)o * (nb * C2) + j * 64 + k]);
   }
   reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);   // bf16 values are exact in fp16
 }
@@ -915,6 +990,14 @@ cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTabl
 cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st) {
   cudaError_t err = launch_tc_gemm(P, W, st);
   if (err != cudaSuccess) return err;
+  if (P.n_edges > 0) {
+    const size_t sm = sizeof(float) * (size_t)P.H * P.L * P.C;
+    err = cudaFuncSetAttribute(logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (err != cudaSuccess) return err;
+    logits_kernel<<<2 * P.grid, 256, sm, st>>>(P);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   switch (P.mmax) {
     case 0: return launch_agg_mm<0>(P, st);
     case 1: return launch_agg_mm<1>(P, st);

@@ -5,7 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-// One GEMM pass over a 128-edge tile: D[128 x n] = A[128 x 64*nk] B[n x 64*nk]^T.
+// One GEMM pass over a 128-edge tile: D[128 x n] = A[128 x 64*nk] B[n x 64*nk]^T.  For a
+// block with |m| = b > 0 the pass covers output rows [n_off, n_off + np) of both y+ and
+// y- (n = 2 np) and B holds only the rows of W_b1 and W_b2 (the sign comes from the
+// instruction's negate-B bit), so each weight is streamed once.
 struct TcPass {
   int kind;          // 0 = radial gate (A = hidden layer), 1 = SO(2) block
   int block;         // |m| of the SO(2) block
@@ -13,6 +16,7 @@ struct TcPass {
   int n_off;         // first output row of the block matrix covered by this pass
   int nk;            // K chunks of 64
   int last_of_kind;  // last gate pass / last pass of block 0
+  int np;            // |m| > 0 blocks: output rows per half; accumulator = [y+ rows | y- rows]
   long long boff;    // byte offset of the pass's first B tile in the prepared image
 };
 

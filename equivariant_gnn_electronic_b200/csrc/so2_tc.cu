@@ -804,10 +804,24 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
   float* Ts = Ds + ((te * P.wfl + 3) & ~3);   // [te][L2][C], 16-byte aligned for float4 reads
   float* Ls = Ts + te * L2 * C;           // [te][nlab]
   const int tid = threadIdx.x, nt = blockDim.x;
+  // small tables in shared memory: lanes index them with different values, which the
+  // parameter (constant) space would serialise
+  __shared__ int s_mult[8], s_lab_off[8], s_shell_l[16], s_shell_off[17], s_orb_shell[32], s_cg_off[128];
+  __shared__ int s_kidx[16 * 16 * 8];
+  for (int x = tid; x < 8; x += nt) {
+    s_mult[x] = Tb.mult[x];
+    s_lab_off[x] = Tb.lab_off[x];
+  }
+  for (int x = tid; x < 16; x += nt) s_shell_l[x] = Tb.shell_l[x];
+  for (int x = tid; x < 17; x += nt) s_shell_off[x] = Tb.shell_off[x];
+  for (int x = tid; x < 32; x += nt) s_orb_shell[x] = Tb.orb_shell[x];
+  for (int x = tid; x < 128; x += nt) s_cg_off[x] = Tb.cg_off[x];
+  for (int x = tid; x < Tb.n_shells * Tb.n_shells * 8; x += nt) s_kidx[x] = Tb.kidx[x];
+  __syncthreads();
   {
     int uo = 0;
     for (int Lq = 0; Lq <= P.lmax; ++Lq) {
-      const int mult = Tb.mult[Lq];
+      const int mult = s_mult[Lq];
       for (int i = tid; i < mult * C; i += nt) {
         const int k = i / C, c = i - k * C;
         Us[uo + c * mult + k] = __bfloat162float(Up.U[Lq][i]);
@@ -859,12 +873,12 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
       const int e = i / nlk;
       int q = i - e * nlk;
       int Lq = 0, uo = 0;
-      while (q >= Tb.mult[Lq]) {
-        q -= Tb.mult[Lq];
-        uo += Tb.mult[Lq] * C;
+      while (q >= s_mult[Lq]) {
+        q -= s_mult[Lq];
+        uo += s_mult[Lq] * C;
         ++Lq;
       }
-      const int k = q, mult = Tb.mult[Lq], nM = 2 * Lq + 1;
+      const int k = q, mult = s_mult[Lq], nM = 2 * Lq + 1;
       const float* U = Us + uo + k;
       const float* t0 = Ts + (e * L2 + Lq * Lq) * C;
       float a[13];
@@ -880,7 +894,7 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
           }
         }
       }
-      float* out = Ls + e * nlab + Tb.lab_off[Lq] + k;
+      float* out = Ls + e * nlab + s_lab_off[Lq] + k;
 #pragma unroll
       for (int M = 0; M < 13; ++M)
         if (M < nM) out[M * mult] = a[M];
@@ -889,15 +903,15 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
     for (int i = tid; i < ne * norb * norb; i += nt) {
       const int e = i / (norb * norb), q = i - e * norb * norb;
       const int ri = q / norb, cj = q - ri * norb;
-      const int a = Tb.orb_shell[ri], b = Tb.orb_shell[cj];
-      const int la = Tb.shell_l[a], lb = Tb.shell_l[b];
-      const int ia = ri - Tb.shell_off[a], jb = cj - Tb.shell_off[b];
+      const int a = s_orb_shell[ri], b = s_orb_shell[cj];
+      const int la = s_shell_l[a], lb = s_shell_l[b];
+      const int ia = ri - s_shell_off[a], jb = cj - s_shell_off[b];
       float v = 0.f;
       for (int Lc = (la > lb ? la - lb : lb - la); Lc <= la + lb; ++Lc) {
-        const int k = Tb.kidx[(a * Tb.n_shells + b) * 8 + Lc];
-        const float* cgm = Tb.cg + Tb.cg_off[(la * 4 + lb) * 8 + Lc] + (ia * (2 * lb + 1) + jb) * (2 * Lc + 1);
-        const float* h = Ls + e * nlab + Tb.lab_off[Lc] + k;
-        const int mult = Tb.mult[Lc];
+        const int k = s_kidx[(a * Tb.n_shells + b) * 8 + Lc];
+        const float* cgm = Tb.cg + s_cg_off[(la * 4 + lb) * 8 + Lc] + (ia * (2 * lb + 1) + jb) * (2 * Lc + 1);
+        const float* h = Ls + e * nlab + s_lab_off[Lc] + k;
+        const int mult = s_mult[Lc];
         for (int M = 0; M < 2 * Lc + 1; ++M) v += cgm[M] * h[M * mult];
       }
       blocks[(e0 + e) * norb * norb + q] = v;

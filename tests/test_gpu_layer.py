@@ -79,7 +79,7 @@ def test_layer_small_bf16_every_atom(egnn):
     check(got, ref, nd, TOL["bf16"])
 
 
-@pytest.mark.parametrize("name", ["hfo2_3000", "gst_8064", "mixed_12000"])
+@pytest.mark.parametrize("name", ["hfo2_3000", "gst_8064", "mixed_12000", "stress_40000"])
 def test_layer_full_size_sampled(egnn, name):
     w = synth.WORKLOADS[name]
     pos, _, _ = cell(name)

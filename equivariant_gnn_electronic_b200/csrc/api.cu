@@ -102,13 +102,20 @@ bool tc_eligible(const egnn_layer_desc* d) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Pass list: radial-gate passes, then the SO(2) blocks |m| = 0..mmax, each block's
-// output rows split into accumulators of at most 512 TMEM columns.
-void tc_plan(const egnn_layer_desc* d, TcParams& P) {
+// output rows split into accumulators of at most 512 TMEM columns.  With `mult`
+// (head, label mode) the output rows of block b are the labels (l >= b, k < mult_l)
+// instead of the channels (l >= b, c < C).  Returns false if the plan needs more
+// passes than TcParams holds.
+bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
   const int L = d->lmax + 1, C = d->channels;
+  const bool label = mult != nullptr;
   P.npass = 0;
+  P.label_mode = label ? 1 : 0;
   long long boff = 0;
-  auto add = [&](int kind, int block, int ntot, int nk) {
+  int roff = 0;
+  auto add = [&](int kind, int block, int ntot, int nk) -> bool {
     for (int off = 0; off < ntot; off += 512) {
+      if (P.npass >= 16) return false;
       TcPass& q = P.pass[P.npass++];
       q.kind = kind;
       q.block = block;
@@ -118,39 +125,64 @@ void tc_plan(const egnn_layer_desc* d, TcParams& P) {
       q.last_of_kind = 0;
       q.np = 0;
       q.boff = boff;
+      q.roff = kind == 1 ? roff : 0;
+      if (kind == 1) roff += q.n;
       boff += (long long)q.n * nk * 128;
     }
     P.pass[P.npass - 1].last_of_kind = 1;
+    return true;
   };
-  add(0, 0, L * 2 * C, C / 64);
+  if (!add(0, 0, L * 2 * C, C / 64)) return false;
   int ycol = 0;
   P.ybase[0] = ycol;
-  add(1, 0, L * C, L * 2 * C / 64);
+  int nr0 = L * C;
+  if (label) {
+    nr0 = 0;
+    for (int l = 0; l < L; ++l) nr0 += mult[l];
+    P.hnr[0] = nr0;
+    P.hroff[0] = roff;
+    nr0 = (nr0 + 31) & ~31;
+  }
+  if (!add(1, 0, nr0, L * 2 * C / 64)) return false;
   ycol += L * C;
   for (int b = 1; b <= d->mmax; ++b) {
     // rows [o0, o0 + np) of y+ and of y-: B = [W_b1 rows ; W_b2 rows] for those outputs,
     // K = the (l, channel) index shared by x+ and x- (each K block feeds 4 MMAs)
-    const int nC = (L - b) * C, kblocks = (L - b) * 2 * C / 64;
+    int nC = (L - b) * C;
+    if (label) {
+      nC = 0;
+      for (int l = b; l < L; ++l) nC += mult[l];
+      P.hnr[b] = nC;
+      P.hroff[b] = roff;
+    }
+    const int kblocks = (L - b) * 2 * C / 64;
     P.ybase[b] = ycol;
-    ycol += 2 * nC;
+    ycol += 2 * (L - b) * C;
     for (int o0 = 0; o0 < nC; o0 += 256) {
+      if (P.npass >= 16) return false;
       TcPass& q = P.pass[P.npass++];
       q.kind = 1;
       q.block = b;
       q.np = nC - o0 < 256 ? nC - o0 : 256;
+      if (label) q.np = (q.np + 15) & ~15;
       q.n = 2 * q.np;
       q.n_off = o0;
       q.nk = kblocks;
       q.last_of_kind = 0;
       q.boff = boff;
+      q.roff = roff;
+      roff += q.n;
       boff += (long long)q.n * kblocks * 128;
     }
   }
   P.ncols_y = ycol;
   P.y0_bytes = L * C * 4;
-  P.y_row_bytes = P.y0_bytes + (ycol - L * C) * 2;
+  P.y_row_bytes = label ? roff * 4 : P.y0_bytes + (ycol - L * C) * 2;
   P.gcols = L * 2 * C;
   P.wprep_bytes = boff;
+  if (label)
+    for (int l = 0; l < 8; ++l) P.mult[l] = l < L ? mult[l] : 0;
+  return true;
 }
 
 struct TcWorkspace {
@@ -175,12 +207,12 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_at
 }
 
 // Fills the tensor-core launch parameters for graph g, weights W and a 1024-aligned
-// workspace; returns false if the workspace is too small.
+// workspace (label mode with `mult`); returns false if the pass plan does not fit.
 bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_desc* desc, const So2Weights& W,
-             const void* node_in, void* node_out, uint8_t* ws, int with_logits) {
+             const void* node_in, void* node_out, uint8_t* ws, int with_logits, const int* mult = nullptr) {
   TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
   memset(&T, 0, sizeof(T));
-  tc_plan(desc, T);
+  if (!tc_plan(desc, T, mult)) return false;
   T.n_atoms = g->n_atoms;
   T.n_edges = g->n_edges;
   T.n_tiles = (int)((g->n_edges + 127) / 128);
@@ -437,9 +469,18 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
   if (use_tc) {
     if (g->n_edges == 0) return EGNN_OK;
     if (((uintptr_t)head_weights | (uintptr_t)node_emb) & 15) return EGNN_ERR_INVALID_ARG;
-    TcParams TP;
+    // Label mode (U^L folded into the SO(2) weights) when its pass plan fits and its
+    // per-edge record is no larger than the channel-space record the workspace holds.
+    TcParams TP, probe;
+    memset(&probe, 0, sizeof(probe));
+    tc_plan(desc, probe);
+    const int y_bytes = probe.y_row_bytes;
+    memset(&probe, 0, sizeof(probe));
+    const bool label = tc_plan(desc, probe, mult) && probe.y_row_bytes <= y_bytes;
     TcWeights TW;
-    fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, 0);
+    if (!fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, 0, label ? mult : nullptr))
+      return EGNN_ERR_UNSUPPORTED;
+    for (int Lc = 0; Lc < 8; ++Lc) TP.U[Lc] = (const __nv_bfloat16*)W.U[Lc];
     HeadUPtrs Up;
     for (int Lc = 0; Lc < 8; ++Lc) Up.U[Lc] = (const __nv_bfloat16*)W.U[Lc];
     if (head_tc_smem_bytes(TP, T.n_lab, 1) > 200 * 1024) return EGNN_ERR_UNSUPPORTED;

@@ -201,7 +201,11 @@ __device__ __forceinline__ void epi_store(const TcParams& P, const TcPass& ps, _
                           pack2h(v[8 * q + 4], v[8 * q + 5]), pack2h(v[8 * q + 6], v[8 * q + 7]));
   } else if (valid) {
     uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
-    if (ps.block == 0) {
+    if (P.label_mode) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + ps.roff + g);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = make_uint4(ru[4 * q], ru[4 * q + 1], ru[4 * q + 2], ru[4 * q + 3]);
+    } else if (ps.block == 0) {
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + col);
 #pragma unroll
       for (int q = 0; q < 8; ++q) dst[q] = make_uint4(ru[4 * q], ru[4 * q + 1], ru[4 * q + 2], ru[4 * q + 3]);
@@ -624,6 +628,24 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
   float v = 0.f;
   if (ps.kind == 0) {
     v = __bfloat162float(W2[(long long)row * C + j * 64 + k]);
+  } else if (P.label_mode) {
+    // the row of label (l, kl) in block b is sum_c U^l[kl, c] * (row (l - b) C + c of
+    // W0, W_b1 or W_b2): the label map applied to the outputs of degree l
+    const int b = ps.block;
+    const bool lower = b > 0 && r >= ps.np;
+    const int lr = ps.n_off + (lower ? r - ps.np : r);
+    if (lr < P.hnr[b]) {
+      int l = b, acc = 0;
+      while (lr >= acc + P.mult[l]) acc += P.mult[l++];
+      const int kl = lr - acc;
+      const __nv_bfloat16* Wb = b == 0 ? W0 : (b == 1 ? (lower ? Wm1b : Wm1a) : (lower ? Wm2b : Wm2a));
+      const long long stride = (long long)(L - b) * C2;
+      const __nv_bfloat16* wcol = Wb + (long long)(l - b) * C * stride + j * 64 + k;
+      const __nv_bfloat16* u = P.U[l] + (long long)kl * C;
+      float a = 0.f;
+      for (int c = 0; c < C; ++c) a += __bfloat162float(u[c]) * __bfloat162float(wcol[c * stride]);
+      v = a;
+    }
   } else if (ps.block == 0) {
     v = __bfloat162float(W0[(long long)row * (L * C2) + j * 64 + k]);
   } else {
@@ -634,7 +656,7 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
     const int o = ps.n_off + (r < ps.np ? r : r - ps.np);
     v = __bfloat162float(W[(long long)o * (nb * C2) + j * 64 + k]);
   }
-  reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);   // bf16 values are exact in fp16
+  reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);   // bf16 values are exact in fp16; label rows round once
 }
 
 // Compile-time layout of kept row r = (l, m) (rows ordered by l, then m = -min(l,MM)..):
@@ -867,6 +889,7 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
         wo += (2 * ml + 1) * (2 * l + 1);
       }
     }
+    __syncthreads();   // the label threads read every channel of t
     // labels: one thread per (edge, L, k) computes every M, so t reads are broadcasts
     // within a warp and U^T reads are consecutive
     for (int i = tid; i < ne * nlk; i += nt) {
@@ -916,6 +939,97 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
       }
       blocks[(e0 + e) * norb * norb + q] = v;
     }
+  }
+}
+
+// Hamiltonian head in label mode.  The SO(2) passes already produced edge-frame labels
+// s[L, m, k] (|m| <= min(L, mmax)); per group of te edges the records and kept Wigner
+// rows are staged in shared memory, the labels are rotated back,
+// h[L, M, k] = sum_m D^L[m, M] s[L, m, k] (one thread per label), and each block entry
+// is the sum of the Clebsch-Gordan images of its shell pair's labels (one thread per
+// entry).  The rotation commutes with U^L because U^L mixes channels only.
+__global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__ TcParams P,
+                                                         const __grid_constant__ HeadTables Tb,
+                                                         float* __restrict__ blocks, int te) {
+  extern __shared__ float hsm[];
+  const int nrec = P.y_row_bytes / 4, wfl4 = (P.wfl + 3) & ~3;
+  const int nlab = Tb.n_lab, norb = Tb.n_orb, mmax = P.mmax;
+  float* Rs = hsm;                 // [te][nrec]
+  float* Ds = Rs + te * nrec;      // [te][wfl4]
+  float* Ls = Ds + te * wfl4;      // [te][nlab]
+  const int tid = threadIdx.x, nt = blockDim.x;
+  __shared__ int s_mult[8], s_lab_off[8], s_woff[8], s_shell_l[16], s_shell_off[17], s_orb_shell[32];
+  __shared__ int s_cg_off[128], s_lb[3][8], s_hroff[3], s_hnr[3];
+  __shared__ int s_kidx[16 * 16 * 8];
+  for (int x = tid; x < 8; x += nt) {
+    s_mult[x] = Tb.mult[x];
+    s_lab_off[x] = Tb.lab_off[x];
+    s_woff[x] = P.woff[x];
+  }
+  for (int x = tid; x < 16; x += nt) s_shell_l[x] = Tb.shell_l[x];
+  for (int x = tid; x < 17; x += nt) s_shell_off[x] = Tb.shell_off[x];
+  for (int x = tid; x < 32; x += nt) s_orb_shell[x] = Tb.orb_shell[x];
+  for (int x = tid; x < 128; x += nt) s_cg_off[x] = Tb.cg_off[x];
+  for (int x = tid; x < Tb.n_shells * Tb.n_shells * 8; x += nt) s_kidx[x] = Tb.kidx[x];
+  if (tid < 3) {
+    s_hroff[tid] = P.hroff[tid];
+    s_hnr[tid] = P.hnr[tid];
+    int acc = 0;   // offset of degree l's labels among block b's rows (l >= b)
+    for (int l = 0; l < 8; ++l) {
+      s_lb[tid][l] = acc;
+      if (l >= tid && l <= P.lmax) acc += P.mult[l];
+    }
+  }
+  const long long e0 = (long long)blockIdx.x * te;
+  const int ne = (int)min((long long)te, P.n_edges - e0);
+  {
+    const float4* rsrc = reinterpret_cast<const float4*>(P.Y + e0 * (long long)P.y_row_bytes);
+    float4* rdst = reinterpret_cast<float4*>(Rs);
+    for (int i = tid; i < ne * nrec / 4; i += nt) rdst[i] = rsrc[i];
+    const float* wsrc = P.wig + e0 * P.wfl;
+    for (int i = tid; i < ne * P.wfl; i += nt) {
+      const int e = i / P.wfl;
+      Ds[e * wfl4 + (i - e * P.wfl)] = wsrc[i];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < ne * nlab; i += nt) {
+    const int e = i / nlab, q0 = i - e * nlab;
+    int q = q0, Lq = 0;
+    while (q >= (2 * Lq + 1) * s_mult[Lq]) {
+      q -= (2 * Lq + 1) * s_mult[Lq];
+      ++Lq;
+    }
+    const int mult = s_mult[Lq], M = q / mult, k = q - M * mult;
+    const int ml = Lq < mmax ? Lq : mmax, dl = 2 * Lq + 1;
+    const float* De = Ds + e * wfl4 + s_woff[Lq] + M;   // row m of D^L at (m + ml) * dl
+    const float* Re = Rs + e * nrec;
+    float h = De[ml * dl] * Re[s_hroff[0] + s_lb[0][Lq] + k];
+    for (int b = 1; b <= ml; ++b) {
+      const int r = s_lb[b][Lq] + k, qq = r >> 8, w = r & 255;
+      const int rest = s_hnr[b] - 256 * qq;
+      const int npq = rest >= 256 ? 256 : ((rest + 15) & ~15);
+      const int base = s_hroff[b] + 512 * qq + w;
+      h += De[(ml + b) * dl] * Re[base] + De[(ml - b) * dl] * Re[base + npq];
+    }
+    Ls[e * nlab + q0] = h;
+  }
+  __syncthreads();
+  for (int i = tid; i < ne * norb * norb; i += nt) {
+    const int e = i / (norb * norb), q = i - e * norb * norb;
+    const int ri = q / norb, cj = q - ri * norb;
+    const int a = s_orb_shell[ri], b = s_orb_shell[cj];
+    const int la = s_shell_l[a], lb = s_shell_l[b];
+    const int ia = ri - s_shell_off[a], jb = cj - s_shell_off[b];
+    float v = 0.f;
+    for (int Lc = (la > lb ? la - lb : lb - la); Lc <= la + lb; ++Lc) {
+      const int k = s_kidx[(a * Tb.n_shells + b) * 8 + Lc];
+      const float* cgm = Tb.cg + s_cg_off[(la * 4 + lb) * 8 + Lc] + (ia * (2 * lb + 1) + jb) * (2 * Lc + 1);
+      const float* h = Ls + e * nlab + s_lab_off[Lc] + k;
+      const int mult = s_mult[Lc];
+      for (int M = 0; M < 2 * Lc + 1; ++M) v += cgm[M] * h[M * mult];
+    }
+    blocks[(e0 + e) * norb * norb + q] = v;
   }
 }
 
@@ -975,6 +1089,20 @@ cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTabl
                            float* blocks, cudaStream_t st) {
   cudaError_t err = launch_tc_gemm(P, W, st);
   if (err != cudaSuccess || P.n_edges == 0) return err;
+  if (P.label_mode) {
+    const int te_max = 16;
+    auto bytes = [&](int t) {
+      return sizeof(float) * (size_t)t * (size_t)(P.y_row_bytes / 4 + ((P.wfl + 3) & ~3) + T.n_lab);
+    };
+    int te = te_max;
+    while (te > 1 && bytes(te) > 100 * 1024) te >>= 1;
+    if (bytes(te) > 200 * 1024) return cudaErrorInvalidValue;
+    err = cudaFuncSetAttribute(head_label_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes(te));
+    if (err != cudaSuccess) return err;
+    const long long groups = (P.n_edges + te - 1) / te;
+    head_label_kernel<<<(unsigned)groups, 256, bytes(te), st>>>(P, T, blocks, te);
+    return cudaGetLastError();
+  }
   int u_total = 0;
   for (int Lq = 0; Lq <= P.lmax; ++Lq) u_total += T.mult[Lq] * P.C;
   int te = 16;   // edges per group; aim at two CTAs per SM (<= 110 KB of shared memory each)

@@ -18,6 +18,7 @@ struct TcPass {
   int last_of_kind;  // last gate pass / last pass of block 0
   int np;            // |m| > 0 blocks: output rows per half; accumulator = [y+ rows | y- rows]
   long long boff;    // byte offset of the pass's first B tile in the prepared image
+  int roff;          // label mode: float offset of the pass's columns in an edge's record
 };
 
 struct TcParams {
@@ -44,6 +45,15 @@ struct TcParams {
   float* Af;                     // attention matrix A[H][L*C] in fp32 (workspace copy)
   int32_t* status;
   int with_logits;               // 1: layer (attention logits from SiLU(y0)); 0: head
+  // Label mode (head only): the SO(2) weights are pre-multiplied by the label maps U^L,
+  // so a pass produces labels in the edge frame, s[l, m, k] = sum_c U^l[k, c] y[l, m, c],
+  // stored in fp32 as the concatenation of the passes' accumulators (record of
+  // y_row_bytes = 4 * sum of pass widths).
+  int label_mode;
+  int hroff[3];                  // record offset of block b's first pass
+  int hnr[3];                    // label rows of block b: sum_{l >= b} mult_l
+  int mult[8];                   // labels per L
+  const __nv_bfloat16* U[8];     // U^L [mult_L][C]
   int npass;
   TcPass pass[16];
   int woff[8];

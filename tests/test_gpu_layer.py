@@ -104,6 +104,24 @@ def test_layer_isolated_atom_keeps_embedding(egnn):
     assert rel_err(out, ref) < TOL["fp32"]
 
 
+@pytest.mark.parametrize("lmax,mmax", [(1, 1), (2, 2), (3, 1), (5, 2), (6, 0)])
+def test_layer_bf16_degrees(egnn, lmax, mmax):
+    # tensor-core layer at the other degree / order limits it accepts, every atom of a
+    # 100-atom HfO2-density cell
+    w = dataclasses.replace(synth.WORKLOADS["hfo2_3000"], lmax=lmax, mmax=mmax)
+    pos, _, box = cell("hfo2_3000", 0, 100)
+    g = gpu_graph(egnn, "hfo2_3000", 0, 100, lmax=lmax, mmax=mmax)
+    desc = egnn.desc_for(w)
+    n = synth.make_embeddings(w, len(pos), 0)
+    W = synth.make_layer_weights(w, 0, bias_std=0.1)
+    out = egnn.layer_forward(g, desc, egnn.pack_weights(W, desc), to_dev(n, torch.bfloat16))
+    torch.cuda.synchronize()
+    assert g.read_status() == 0
+    rp, src, sh = oracle_graph("hfo2_3000", 0, 100)
+    ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
+    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"])
+
+
 def test_layer_is_deterministic(egnn):
     w = synth.WORKLOADS["hfo2_3000"]
     pos, species, box = cell("hfo2_3000", 0, 300)
@@ -147,6 +165,30 @@ def test_head_full_size_sampled(egnn, name):
     w = synth.WORKLOADS[name]
     pos, _, _ = cell(name)
     got, ref = run_head(egnn, name, w, atoms=sample_atoms(len(pos), 4, 5))
+    assert rel_err(got, ref) < TOL["bf16"]
+
+
+def test_head_bf16_every_edge(egnn):
+    # tensor-core head, labels folded into the SO(2) weights, every edge of a 150-atom cell
+    w = synth.WORKLOADS["hfo2_3000"]
+    got, ref = run_head(egnn, "hfo2_3000", w, n_atoms=150, bias_std=0.1)
+    assert rel_err(got, ref) < TOL["bf16"]
+
+
+def test_head_bf16_wide_template(egnn):
+    # 8 s + 8 p shells (32 orbitals): 384 label rows for |m| = 0 and 256 per half for
+    # |m| = 1, i.e. a full 512-column accumulator
+    w = synth.WORKLOADS["hfo2_3000"]
+    shells = (0,) * 8 + (1,) * 8
+    got, ref = run_head(egnn, "hfo2_3000", w, n_atoms=120, bias_std=0.1, shells=shells)
+    assert rel_err(got, ref) < TOL["bf16"]
+
+
+def test_head_bf16_channel_space(egnn):
+    # lmax 2 with ten p shells: the label record (960 floats) is larger than the
+    # channel-space record (768), so the head rotates y back per channel instead
+    w = dataclasses.replace(synth.WORKLOADS["hfo2_3000"], lmax=2, shells=(1,) * 10)
+    got, ref = run_head(egnn, "hfo2_3000", w, n_atoms=120, bias_std=0.1)
     assert rel_err(got, ref) < TOL["bf16"]
 
 

@@ -175,6 +175,15 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
       boff += (long long)q.n * kblocks * 128;
     }
   }
+  // A tiles of one edge tile for the split pipeline: block 0 one per (l, 64 channels),
+  // |m| = b > 0 an x+ / x- pair per (l >= b, 64 channels)
+  const int kpl = 2 * C / 64;
+  P.xbase[0] = 0;
+  P.nch = L * kpl;
+  for (int b = 1; b <= d->mmax; ++b) {
+    P.xbase[b] = P.nch;
+    P.nch += 2 * (L - b) * kpl;
+  }
   P.ncols_y = ycol;
   P.y0_bytes = L * C * 4;
   P.y_row_bytes = label ? roff * 4 : P.y0_bytes + (ycol - L * C) * 2;
@@ -186,7 +195,7 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
 }
 
 struct TcWorkspace {
-  size_t wprep, gate, y, logits, node_h, af, total;
+  size_t wprep, gate, x, y, logits, node_h, af, total;
 };
 
 TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_atoms) {
@@ -195,9 +204,11 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_at
   tc_plan(d, P);
   TcWorkspace w;
   size_t E = n_edges > 0 ? (size_t)n_edges : 0;
+  const size_t tch = (size_t)tc_chunk_tiles((int)((E + 127) / 128));
   w.wprep = 0;
   w.gate = align_up((size_t)P.wprep_bytes, 1024);
-  w.y = w.gate + align_up((size_t)kTcMaxGrid * 128 * P.gcols * 2, 1024);
+  w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
+  w.y = w.x + align_up(tch * P.nch * 16384, 1024);
   w.logits = w.y + align_up(E * (size_t)P.y_row_bytes, 1024);
   w.node_h = w.logits + align_up(E * d->heads * 4, 1024);
   size_t N = n_atoms > 0 ? (size_t)n_atoms : 0;
@@ -244,7 +255,9 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   T.A = (const __nv_bfloat16*)W.A;
   T.bA = (const __nv_bfloat16*)W.bA;
   T.wprep = ws + wl.wprep;
-  T.gate_scratch = (__half*)(ws + wl.gate);
+  T.gates = (__half*)(ws + wl.gate);
+  T.gate_scratch = T.gates;
+  T.X = ws + wl.x;
   T.Y = ws + wl.y;
   T.logits = (float*)(ws + wl.logits);
   T.node_h = (__half*)(ws + wl.node_h);

@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     // ---------------- B loader ----------------
     if (lane == 0) {
       uint32_t ib = 0;
-      for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x) {
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
         for (int p = 0; p < P.npass && !*abort; ++p) {
           const TcPass& ps = P.pass[p];
           const uint32_t bytes = (uint32_t)ps.n * 128u;
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t ia = 0, ib = 0, ip = 0, it = 0;
-      for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x, ++it) {
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
         bool hid_waited = false;
         for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
           const TcPass& ps = P.pass[p];
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     const int q = pidx & 7;                    // 16-byte chunk within a 64-channel slice
     const int rb = pidx >> 3;                  // 0..31
     uint32_t ia = 0, it = 0;
-    for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x, ++it) {
+    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
       int srcs[4], dsts[4];
       float dists[4];
       bool valids[4];
@@ -571,11 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
-    __half* gsc = P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
     uint32_t ip = 0;
-    for (int t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x) {
+    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
       const long long e = (long long)t * 128 + r;
       const bool valid = e < E;
+      __half* gsc = P.gates ? P.gates + ((long long)(t - P.t_begin) * 128 + r) * P.gcols
+                            : P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
         if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full), ip & 1, P.status, abort, 256)) break;
@@ -1033,6 +1034,293 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
   }
 }
 
+
+// ---------------- rotate + gate: the A operands of the SO(2) GEMM ----------------
+// One CTA per 128-edge tile.  For every edge and degree l the kept rows of the edge
+// frame, x[l, m, :] = g[l, :] * sum_{m'} D^l[m, m'] [n_s || n_d][l, m', :] for
+// |m| <= min(l, mmax), are computed with packed fp16 FMAs from the fp16 copy of the
+// node table and written straight into the 128-byte-swizzled K-major 128 x 64 tiles
+// that the GEMM's bulk copies move (16-byte piece c of row r at position c ^ (r & 7)).
+// Warp = one edge at a time, lane = one 8-channel piece of the 256-wide pair row
+// (lanes 0-15 the source atom, 16-31 the destination): a node row is one 512-byte
+// warp load, an A row four full 128-byte lines.  All 2l+1 rows of n[l] are loaded
+// before the FMAs, which keeps up to 13 x 16 B per lane in flight.
+template <int LM, int MM>
+__global__ void __launch_bounds__(256) rotate_kernel(const __grid_constant__ TcParams P) {
+  constexpr int L = LM + 1;
+  __shared__ int s_node[2][128];   // source and destination atom of each row
+  const int t = P.t_begin + blockIdx.x;
+  const long long E = P.n_edges;
+  if (threadIdx.x < 128) {
+    const int r = threadIdx.x;
+    const long long e = (long long)t * 128 + r;
+    int sv = 0, dv = 0;
+    if (e < E) {
+      sv = P.src[e];
+      int lo = 0, hi = P.n_atoms;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+      }
+      dv = lo;
+      if (sv < 0 || sv >= P.n_atoms) {
+        egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
+        sv = dv;
+      }
+    }
+    s_node[0][r] = sv;
+    s_node[1][r] = dv;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int side = lane >> 4, cs = lane >> 3, qq = lane & 7;
+  uint8_t* xt = P.X + (long long)blockIdx.x * P.nch * 16384;
+  for (int r = warp; r < 128; r += 8) {
+    const long long e = (long long)t * 128 + r;
+    const bool valid = e < E;
+    const __half* zn = P.node_h + (long long)s_node[side][r] * (L * L) * 128 + (lane & 15) * 8;
+    const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl;
+    const __half* gr = P.gates + ((long long)blockIdx.x * 128 + r) * P.gcols + lane * 8;
+    uint8_t* xr = xt + r * 128 + ((qq ^ (r & 7)) << 4);
+    int wo = 0;
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+      const int dl = 2 * l + 1, ml = l < MM ? l : MM, nr = 2 * ml + 1;
+      // the nr x dl kept coefficients of D^l, spread over the lanes as fp16 pairs
+      uint32_t cf[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const int idx = lane + 32 * k;
+        const float v = (valid && idx < nr * dl) ? __ldg(De + wo + idx) : 0.f;
+        const __half2 h = __float2half2_rn(v);
+        cf[k] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      uint4 zq[2 * LM + 1];
+#pragma unroll
+      for (int mp = 0; mp < dl; ++mp)
+        zq[mp] = valid ? __ldg(reinterpret_cast<const uint4*>(zn + (l * l + mp) * 128)) : make_uint4(0, 0, 0, 0);
+      const uint4 gq = valid ? __ldg(reinterpret_cast<const uint4*>(gr + l * 256)) : make_uint4(0, 0, 0, 0);
+      __half2 acc[2 * MM + 1][4];
+#pragma unroll
+      for (int m = 0; m < nr; ++m)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][i] = __float2half2_rn(0.f);
+#pragma unroll
+      for (int mp = 0; mp < dl; ++mp) {
+        const __half2* zh = reinterpret_cast<const __half2*>(&zq[mp]);
+#pragma unroll
+        for (int m = 0; m < nr; ++m) {
+          const int k = m * dl + mp;
+          const uint32_t cu = __shfl_sync(0xffffffffu, cf[k >> 5], k & 31);
+          const __half2 c = *reinterpret_cast<const __half2*>(&cu);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[m][i] = __hfma2(c, zh[i], acc[m][i]);
+        }
+      }
+      const __half2* gh = reinterpret_cast<const __half2*>(&gq);
+#pragma unroll
+      for (int m = 0; m < nr; ++m) {
+        const int mm = m - ml, b = mm < 0 ? -mm : mm;
+        const int id = b == 0 ? l * 4 + cs : P.xbase[b] + ((l - b) * 4 + cs) * 2 + (mm < 0 ? 1 : 0);
+        uint4 w;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __half2 x = __hmul2(acc[m][i], gh[i]);
+          pw[i] = *reinterpret_cast<const uint32_t*>(&x);
+        }
+        *reinterpret_cast<uint4*>(xr + (long long)id * 16384) = w;
+      }
+      wo += nr * dl;
+    }
+  }
+}
+
+// ---------------- SO(2) GEMM: bulk-copied A and B, tcgen05, TMEM epilogue ----------------
+// Persistent over the tiles of a range.  Warp 0 bulk-copies the prepared A tiles of
+// the rotate kernel and the weight tiles, warp 1 issues the MMAs (one thread) and
+// owns TMEM, warps 2-5 drain each pass's accumulator (thread = TMEM lane = edge).
+constexpr int kGA = 6;                 // A stages (16 KB each)
+constexpr int kGThreads = 6 * 32;
+
+struct GemmCtl {
+  uint64_t a_full[kGA], a_empty[kGA], b_full[kSB], b_empty[kSB];
+  uint64_t acc_full, acc_empty, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(base + kGA * kAStage + kSB * kBStage);
+  const uint32_t A_u32 = base_u32;
+  const uint32_t B_u32 = base_u32 + kGA * kAStage;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &ctl->abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGA; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->a_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->a_empty[i]), 1);
+    }
+    for (int i = 0; i < kSB; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->b_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->b_empty[i]), 1);
+    }
+    tc::mbar_init(tc::smem_u32(&ctl->acc_full), 1);
+    tc::mbar_init(tc::smem_u32(&ctl->acc_empty), 128);
+    tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
+    ctl->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(&ctl->tmem_base), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const long long E = P.n_edges;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t ia = 0, ib = 0;
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
+        const uint8_t* xt = P.X + (long long)(t - P.t_begin) * P.nch * 16384;
+        for (int p = 0; p < P.npass && !*abort; ++p) {
+          const TcPass& ps = P.pass[p];
+          const uint32_t bytes = (uint32_t)ps.n * 128u;
+          const int na = ps.block > 0 ? 2 : 1;
+          for (int kb = 0; kb < ps.nk && !*abort; ++kb, ++ib) {
+            const int sb = ib % kSB;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kSB) & 1) ^ 1, P.status, abort, 64)) break;
+            tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->b_full[sb]), bytes);
+            tc::bulk_g2s(B_u32 + sb * kBStage, P.wprep + ps.boff + (long long)kb * bytes, bytes,
+                         tc::smem_u32(&ctl->b_full[sb]));
+            for (int h = 0; h < na; ++h, ++ia) {
+              const int sa = ia % kGA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa]), ((ia / kGA) & 1) ^ 1, P.status, abort, 64)) break;
+              const int id = ps.block == 0 ? kb : P.xbase[ps.block] + 2 * kb + h;
+              tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->a_full[sa]), (uint32_t)kAStage);
+              tc::bulk_g2s(A_u32 + sa * kAStage, xt + (long long)id * kAStage, (uint32_t)kAStage,
+                           tc::smem_u32(&ctl->a_full[sa]));
+            }
+          }
+        }
+      }
+      // the newest phase of every stage must have landed before the CTA exits
+      for (uint32_t k = (ib > (uint32_t)kSB ? ib - kSB : 0); k < ib; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kSB]);
+        const uint64_t t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(bar, (k / kSB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        }
+      }
+      for (uint32_t k = (ia > (uint32_t)kGA ? ia - kGA : 0); k < ia; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->a_full[k % kGA]);
+        const uint64_t t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(bar, (k / kGA) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t ia = 0, ib = 0, ip = 0;
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
+        for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
+          const TcPass& ps = P.pass[p];
+          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty), (ip & 1) ^ 1, P.status, abort, 32)) break;
+          tc::tc_fence_after();
+          if (ps.block > 0) {
+            // y+ += x+ W1^T - x- W2^T ; y- += x+ W2^T + x- W1^T, one K block of 64 per step
+            const int np = ps.np;
+            const uint32_t idn = tc::idesc_f16(128, np), idneg = tc::idesc_f16(128, np, true);
+            for (int kb = 0; kb < ps.nk; ++kb, ++ib, ia += 2) {
+              const int sb = ib % kSB, sp = ia % kGA, sm = (ia + 1) % kGA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sp]), (ia / kGA) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sm]), ((ia + 1) / kGA) & 1, P.status, abort)) break;
+              tc::tc_fence_after();
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ap = tc::sw128_desc(A_u32 + sp * kAStage + ks * 32);
+                const uint64_t am = tc::sw128_desc(A_u32 + sm * kAStage + ks * 32);
+                const uint64_t b1 = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
+                const uint64_t b2 = tc::sw128_desc(B_u32 + sb * kBStage + np * 128 + ks * 32);
+                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                tc::mma_bf16(tmem, ap, b1, idn, acc);
+                tc::mma_bf16(tmem, am, b2, idneg, 1u);
+                tc::mma_bf16(tmem + np, ap, b2, idn, acc);
+                tc::mma_bf16(tmem + np, am, b1, idn, 1u);
+              }
+              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sp]));
+              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sm]));
+              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
+            }
+          } else {
+            for (int kb = 0; kb < ps.nk; ++kb, ++ib, ++ia) {
+              const int sb = ib % kSB, sa = ia % kGA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sa]), (ia / kGA) & 1, P.status, abort)) break;
+              tc::tc_fence_after();
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = tc::sw128_desc(A_u32 + sa * kAStage + ks * 32);
+                for (int n0 = 0; n0 < ps.n; n0 += 256) {
+                  const int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
+                  const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + n0 * 128 + ks * 32);
+                  tc::mma_bf16(tmem + n0, ad, bd, tc::idesc_f16(128, ns), (kb > 0 || ks > 0) ? 1u : 0u);
+                }
+              }
+              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
+              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
+            }
+          }
+          tc::mma_commit(tc::smem_u32(&ctl->acc_full));
+        }
+      }
+      // every issued MMA must finish before TMEM is released
+      tc::mma_commit(tc::smem_u32(&ctl->mma_done));
+      const uint64_t t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(tc::smem_u32(&ctl->mma_done), 0) && tc::globaltimer() - t0 < 2000000000ull) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: thread = TMEM lane = edge ----------------
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
+    uint32_t ip = 0;
+    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
+      const long long e = (long long)t * 128 + r;
+      const bool valid = e < E;
+      for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
+        const TcPass& ps = P.pass[p];
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full), ip & 1, P.status, abort, 128)) break;
+        tc::tc_fence_after();
+        for (int g = 0; g < ps.n; g += 32) {
+          uint32_t ra[32];
+          tc::tmem_ld32_issue(tl + g, ra);
+          tc::tmem_ld_wait(ra);
+          epi_store(P, ps, nullptr, e, valid, g, ra);
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty));
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 }  // namespace
 
 size_t so2_tc_smem_bytes() { return kSA * kAStage + kSB * kBStage + kHStage + sizeof(SmemCtl) + 1024; }
@@ -1057,6 +1345,29 @@ __global__ void a_to_f32_kernel(const __nv_bfloat16* __restrict__ A, float* __re
   if (i < n) out[i] = __bfloat162float(A[i]);
 }
 
+template <int LM, int MM>
+static void launch_rotate(const TcParams& P, int nt, cudaStream_t st) {
+  rotate_kernel<LM, MM><<<nt, 256, 0, st>>>(P);
+}
+
+static cudaError_t launch_rotate_any(const TcParams& P, int nt, cudaStream_t st) {
+  switch (P.mmax * 8 + P.lmax) {
+#define EGNN_ROT_CASE(LMv, MMv) \
+  case MMv * 8 + LMv:          \
+    launch_rotate<LMv, MMv>(P, nt, st); \
+    break;
+    EGNN_ROT_CASE(1, 0) EGNN_ROT_CASE(2, 0) EGNN_ROT_CASE(3, 0) EGNN_ROT_CASE(4, 0) EGNN_ROT_CASE(5, 0)
+    EGNN_ROT_CASE(6, 0) EGNN_ROT_CASE(1, 1) EGNN_ROT_CASE(2, 1) EGNN_ROT_CASE(3, 1) EGNN_ROT_CASE(4, 1)
+    EGNN_ROT_CASE(5, 1) EGNN_ROT_CASE(6, 1) EGNN_ROT_CASE(2, 2) EGNN_ROT_CASE(3, 2) EGNN_ROT_CASE(4, 2)
+    EGNN_ROT_CASE(5, 2) EGNN_ROT_CASE(6, 2)
+#undef EGNN_ROT_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Weight prep, then per range of edge tiles: gate GEMM -> rotate -> SO(2) GEMM.
 static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStream_t st) {
   if (P.with_logits) {
     const int na = P.H * P.L * P.C;
@@ -1069,14 +1380,34 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
                                                                       W.Wm[1][0], W.Wm[1][1], total,
                                                                       const_cast<uint8_t*>(P.wprep));
   cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  if (P.n_edges > 0) {
-    size_t sm = so2_tc_smem_bytes();
-    err = cudaFuncSetAttribute(so2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (err != cudaSuccess) return err;
-    so2_tc_kernel<<<P.grid, kThreads, sm, st>>>(P);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+  if (err != cudaSuccess || P.n_edges == 0) return err;
+  // split the pass list: gate passes (kind 0) lead, SO(2) passes follow
+  TcParams Pg = P, Ps = P;
+  int ng = 0;
+  while (ng < P.npass && P.pass[ng].kind == 0) ++ng;
+  Pg.npass = ng;
+  Ps.npass = P.npass - ng;
+  for (int i = 0; i < Ps.npass; ++i) Ps.pass[i] = P.pass[ng + i];
+  const size_t sm_g = so2_tc_smem_bytes();
+  const size_t sm_s = kGA * kAStage + kSB * kBStage + sizeof(GemmCtl) + 1024;
+  if ((err = cudaFuncSetAttribute(so2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) !=
+      cudaSuccess)
+    return err;
+  if ((err = cudaFuncSetAttribute(so2_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_s)) !=
+      cudaSuccess)
+    return err;
+  const int tch = tc_chunk_tiles(P.n_tiles);
+  for (int tb = 0; tb < P.n_tiles; tb += tch) {
+    const int te = tb + tch < P.n_tiles ? tb + tch : P.n_tiles;
+    const int nt = te - tb;
+    const int grid = P.grid < nt ? P.grid : nt;
+    Pg.t_begin = Ps.t_begin = tb;
+    Pg.t_end = Ps.t_end = te;
+    so2_tc_kernel<<<grid, kThreads, sm_g, st>>>(Pg);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = launch_rotate_any(Ps, nt, st)) != cudaSuccess) return err;
+    so2_gemm_kernel<<<grid, kGThreads, sm_s, st>>>(Ps);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   return cudaSuccess;
 }

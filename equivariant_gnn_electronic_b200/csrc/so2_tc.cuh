@@ -54,6 +54,16 @@ struct TcParams {
   int hnr[3];                    // label rows of block b: sum_{l >= b} mult_l
   int mult[8];                   // labels per L
   const __nv_bfloat16* U[8];     // U^L [mult_L][C]
+  // Tile range of one launch and the per-range buffers of the split pipeline
+  // (gate GEMM -> rotate -> SO(2) GEMM): gates of the range's rows in fp16, and the
+  // rotated, gated A operands as 128 x 64 fp16 tiles in the 128-byte-swizzled
+  // K-major image the MMA reads, `nch` tiles per edge tile, block b's first at
+  // xbase[b] (a |m| > 0 K block stores x+ then x-).
+  int t_begin, t_end;
+  __half* gates;                 // [(t_end - t_begin) * 128][gcols]
+  uint8_t* X;                    // [(t_end - t_begin)][nch][128 * 128 B]
+  int nch;
+  int xbase[3];
   int npass;
   TcPass pass[16];
   int woff[8];
@@ -66,6 +76,14 @@ struct TcWeights {
 };
 
 constexpr int kTcMaxGrid = 160;
+constexpr int kTcChunkTiles = 4096;   // edge tiles per launch range (bounds the gate and A buffers)
+
+// Tiles per launch range: the fewest ranges of at most kTcChunkTiles, balanced.
+inline int tc_chunk_tiles(int n_tiles) {
+  if (n_tiles <= 0) return 1;
+  const int nr = (n_tiles + kTcChunkTiles - 1) / kTcChunkTiles;
+  return (n_tiles + nr - 1) / nr;
+}
 
 struct HeadTables;
 struct HeadUPtrs {

@@ -114,12 +114,13 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
   long long boff = 0;
   int roff = 0;
   auto add = [&](int kind, int block, int ntot, int nk) -> bool {
-    for (int off = 0; off < ntot; off += 512) {
+    const int step = kind == 0 ? 256 : 512;   // gate passes alternate two 256-column accumulators
+    for (int off = 0; off < ntot; off += step) {
       if (P.npass >= 16) return false;
       TcPass& q = P.pass[P.npass++];
       q.kind = kind;
       q.block = block;
-      q.n = ntot - off < 512 ? ntot - off : 512;
+      q.n = ntot - off < step ? ntot - off : step;
       q.n_off = off;
       q.nk = nk;
       q.last_of_kind = 0;
@@ -256,7 +257,6 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   T.bA = (const __nv_bfloat16*)W.bA;
   T.wprep = ws + wl.wprep;
   T.gates = (__half*)(ws + wl.gate);
-  T.gate_scratch = T.gates;
   T.X = ws + wl.x;
   T.Y = ws + wl.y;
   T.logits = (float*)(ws + wl.logits);

@@ -11,26 +11,24 @@
 // here the contractions that are GEMMs run on tcgen05 and the small per-edge
 // rotations stay on the CUDA cores that feed them.
 //
-// Three launches per layer:
+// Launches per layer (C = 128, bf16 storage, fp16 operands, fp32 accumulation):
 //   prep_weights  packs the gate and SO(2) weight matrices into the exact
 //                 shared-memory image of K-major 128-byte-swizzled B tiles, one
-//                 tile per (pass, 64-wide K chunk), so one 1-D bulk copy moves it.
-//   so2_tc        persistent; per tile of 128 consecutive edges (one edge per
-//                 TMEM lane) it runs a list of passes, each a GEMM
-//                 D[128 x N<=512] = A[128 x K] B[N x K]^T accumulated in TMEM:
-//                   gate passes  A = SiLU(W1 rho(|r_e|) + b1), B = W2 -> gate g_e
-//                                (+ b2, bf16) into a per-CTA scratch;
-//                   SO(2) passes A = g_e * (D^l(R_e) [n_s || n_d]) rows |m| = b
-//                                built on the fly, B = W0 (b = 0) or the real
-//                                form [[W_b1, -W_b2], [W_b2, W_b1]] (b > 0)
-//                                -> y_e (bf16).
-//                 Warp roles: 0 bulk-copies B tiles, 1 issues MMAs (one thread)
-//                 and owns TMEM, 2-9 build A tiles (8 lanes per 128-byte row slice so
-//                 that gathers are coalesced), 10-13 drain TMEM.
-//   agg           one CTA per destination atom, thread = channel pair: attention
-//                 logits from SiLU(y0), online softmax over the atom's incoming
-//                 edges, rotate y back with the kept rows of D^l(R_e), weighted
-//                 sum, residual; no atomics.
+//                 tile per (pass, 64-wide K chunk), so one 1-D bulk copy moves it
+//                 (head: the label maps U^L are folded into the SO(2) rows here);
+//   to_f16        exact fp16 copy of the node table for the rotation.
+//   Then per range of at most 4096 edge tiles (128 edges each):
+//   gate          g_e = W2 SiLU(W1 rho(|r_e|) + b1) + b2 on tcgen05 (hidden layer on
+//                 the CUDA cores), fp16 per edge;
+//   rotate        x_e = g_e * (D^l(R_e) [n_s || n_d]) for the kept rows |m| <= mmax,
+//                 written as ready-made A tiles;
+//   so2_gemm      D[128 x N <= 512] = A[128 x K] B[N x K]^T per pass in TMEM, with
+//                 B = W0 (|m| = 0) or [W_b1 ; W_b2] read by four MMAs, one with the
+//                 negate-B bit, per K block (|m| = b > 0); the epilogue writes y_e
+//                 (y0 in fp32, |m| > 0 in bf16) or, for the head, edge-frame labels.
+//   Then logits (attention logits from SiLU(y0)) and agg (one CTA per destination
+//   atom: softmax over its incoming edges, rotate back with the kept rows of D^l,
+//   weighted sum, residual; no atomics).
 #include <math.h>
 
 #include "common.cuh"
@@ -40,20 +38,18 @@
 
 namespace {
 
-constexpr int kSA = 4;                 // A stages (128 x 64 bf16 = 16 KB each)
-constexpr int kSB = 2;                 // B stages (<= 512 x 64 bf16 = 64 KB each)
-constexpr int kAStage = 128 * 128;
+constexpr int kSB = 2;                 // B stages (<= 512 x 64 fp16 = 64 KB each)
+constexpr int kAStage = 128 * 128;     // one 128 x 64 fp16 A tile (16 KB)
 constexpr int kBStage = 512 * 128;
-constexpr int kPW = 8;                         // producer warps (256 threads: 8 lanes per row, 32 rows per step)
-constexpr int kProducers = kPW * 32;
-constexpr int kThreads = (2 + kPW + 4) * 32;   // 0 loader, 1 MMA, producers, 4 epilogue warps
 constexpr int kTmemCols = 512;
+constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = C = 128: two A tiles
+constexpr int kPW = 8;                 // gate kernel: warps computing the hidden layer
+constexpr int kProducers = kPW * 32;
+constexpr int kThreads = (2 + kPW + 4) * 32;   // 0 loader, 1 MMA, hidden layer, 4 epilogue warps
 
-constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = 128: 2 chunks
-
-struct SmemCtl {
-  uint64_t a_full[kSA], a_empty[kSA], b_full[kSB], b_empty[kSB];
-  uint64_t acc_full, acc_empty, gate_ready, mma_done, hid_full, hid_empty;
+struct GateCtl {
+  uint64_t b_full[kSB], b_empty[kSB], acc_full[2], acc_empty[2];
+  uint64_t hid_full, hid_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -72,113 +68,9 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Producer helpers.  A thread owns NCH consecutive fp16 channels (NCH / 2 half2) of one
-// tile row.  acc (+)= sum_{mp < dl} co[mp] * z[mp * C + channels] in packed fp16
-// (one HFMA2 per channel pair and row); BATCH rows of z are loaded before their FMAs.
-template <int NCH, int BATCH>
-__device__ __forceinline__ void rot_h1(__half2* acc, const __half* z, int C, const float* co, int dl) {
-  constexpr int Q = NCH / 8;                 // 16-byte loads per row
-  for (int mp0 = 0; mp0 < dl; mp0 += BATCH) {
-    uint4 q[BATCH][Q];
-    __half2 c[BATCH];
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      const bool ok = mp0 + u < dl;
-      const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
-#pragma unroll
-      for (int k = 0; k < Q; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
-      c[u] = __float2half2_rn(ok ? __ldg(co + mp0 + u) : 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u)
-#pragma unroll
-      for (int k = 0; k < Q; ++k) {
-        const __half2* h = reinterpret_cast<const __half2*>(&q[u][k]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[4 * k + i] = __hfma2(c[u], h[i], acc[4 * k + i]);
-      }
-  }
-}
-
-// Same for the two coefficient rows of the (+b, -b) pair, which share z.
-template <int NCH, int BATCH>
-__device__ __forceinline__ void rot_h2(__half2* ap, __half2* am, const __half* z, int C, const float* cop,
-                                       const float* com, int dl) {
-  constexpr int Q = NCH / 8;
-  for (int mp0 = 0; mp0 < dl; mp0 += BATCH) {
-    uint4 q[BATCH][Q];
-    __half2 cp[BATCH], cm[BATCH];
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      const bool ok = mp0 + u < dl;
-      const uint4* zp = reinterpret_cast<const uint4*>(z + (ok ? mp0 + u : 0) * C);
-#pragma unroll
-      for (int k = 0; k < Q; ++k) q[u][k] = ok ? __ldg(zp + k) : make_uint4(0, 0, 0, 0);
-      cp[u] = __float2half2_rn(ok ? __ldg(cop + mp0 + u) : 0.f);
-      cm[u] = __float2half2_rn(ok ? __ldg(com + mp0 + u) : 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u)
-#pragma unroll
-      for (int k = 0; k < Q; ++k) {
-        const __half2* h = reinterpret_cast<const __half2*>(&q[u][k]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          ap[4 * k + i] = __hfma2(cp[u], h[i], ap[4 * k + i]);
-          am[4 * k + i] = __hfma2(cm[u], h[i], am[4 * k + i]);
-        }
-      }
-  }
-}
-
-// acc *= g for the thread's NCH fp16 channels read from the gate scratch.
-template <int NCH>
-__device__ __forceinline__ void gate_mul(__half2* acc, const __half* g) {
-  const uint4* gp = reinterpret_cast<const uint4*>(g);
-#pragma unroll
-  for (int k = 0; k < NCH / 8; ++k) {
-    const uint4 w = gp[k];
-    const __half2* h = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[4 * k + i] = __hmul2(acc[4 * k + i], h[i]);
-  }
-}
-
-// Writes NCH fp16 values (NCH / 2 half2) as columns [NCH*part, NCH*part + NCH) of row r of a
-// 128B-swizzled K-major tile (16-byte chunk c of row r sits at position c ^ (r & 7)).
-template <int NCH>
-__device__ __forceinline__ void store_row_h(uint8_t* tile, int r, int part, const __half2* v) {
-#pragma unroll
-  for (int q = 0; q < NCH / 8; ++q) {
-    const int chunk = part * (NCH / 8) + q;
-    uint4 w;
-    w.x = *reinterpret_cast<const uint32_t*>(&v[4 * q + 0]);
-    w.y = *reinterpret_cast<const uint32_t*>(&v[4 * q + 1]);
-    w.z = *reinterpret_cast<const uint32_t*>(&v[4 * q + 2]);
-    w.w = *reinterpret_cast<const uint32_t*>(&v[4 * q + 3]);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
-  }
-}
-
 __device__ __forceinline__ uint32_t pack2h(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// Writes NCH fp32 values, rounded to fp16, as columns [NCH*part, NCH*part + NCH) of row r
-// of a 128B-swizzled K-major tile.
-template <int NCH>
-__device__ __forceinline__ void store_row_f(uint8_t* tile, int r, int part, const float* v) {
-#pragma unroll
-  for (int q = 0; q < NCH / 8; ++q) {
-    const int chunk = part * (NCH / 8) + q;
-    uint4 w;
-    w.x = pack2h(v[8 * q + 0], v[8 * q + 1]);
-    w.y = pack2h(v[8 * q + 2], v[8 * q + 3]);
-    w.z = pack2h(v[8 * q + 4], v[8 * q + 5]);
-    w.w = pack2h(v[8 * q + 6], v[8 * q + 7]);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
-  }
 }
 
 // Epilogue store of one 32-column group of a pass (thread = edge row): gate passes
@@ -260,38 +152,46 @@ __global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcP
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_constant__ TcParams P) {
+// Radial gate GEMM, persistent over the tiles of a range: per 128-edge tile the
+// hidden layer h = SiLU(W1 rho(|r_e|) + b1) (K Gaussians) is computed on the CUDA
+// cores from W1 staged in shared memory and written as two 128 x 64 fp16 A tiles; the
+// gate passes g = h W2^T (+ b2 in the epilogue) run on tcgen05 into two 256-column
+// TMEM accumulators used alternately, so one pass drains while the next accumulates.
+// Gates are written per edge in fp16.  Warp 0 bulk-copies W2 tiles, warp 1 issues
+// the MMAs and owns TMEM, warps 2-9 compute the hidden layer (8 lanes per 128-byte row
+// slice, 4 rows per thread), warps 10-13 drain (thread = TMEM lane = edge).
+__global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
-  uint8_t* Abuf = base;
-  uint8_t* Bbuf = base + kSA * kAStage;
-  uint8_t* Hbuf = Bbuf + kSB * kBStage;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(Hbuf + kHStage);
-  const uint32_t A_u32 = base_u32;
-  const uint32_t B_u32 = base_u32 + kSA * kAStage;
-  const uint32_t H_u32 = B_u32 + kSB * kBStage;
+  uint8_t* Hbuf = base + kSB * kBStage;
+  float* W1s = reinterpret_cast<float*>(Hbuf + kHStage);   // [K][C] fp32
+  GateCtl* ctl = reinterpret_cast<GateCtl*>(W1s + P.K * P.C);
+  const uint32_t B_u32 = base_u32;
+  const uint32_t H_u32 = base_u32 + kSB * kBStage;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &ctl->abort;
+  const int C = P.C, K = P.K;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSA; ++i) {
-      tc::mbar_init(tc::smem_u32(&ctl->a_full[i]), kProducers);
-      tc::mbar_init(tc::smem_u32(&ctl->a_empty[i]), 1);
-    }
     for (int i = 0; i < kSB; ++i) {
       tc::mbar_init(tc::smem_u32(&ctl->b_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->b_empty[i]), 1);
     }
-    tc::mbar_init(tc::smem_u32(&ctl->acc_full), 1);
-    tc::mbar_init(tc::smem_u32(&ctl->acc_empty), 128);
-    tc::mbar_init(tc::smem_u32(&ctl->gate_ready), 128);
-    tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->acc_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->acc_empty[i]), 128);
+    }
     tc::mbar_init(tc::smem_u32(&ctl->hid_full), kProducers);
     tc::mbar_init(tc::smem_u32(&ctl->hid_empty), 1);
+    tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
     ctl->abort = 0;
     tc::fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < C * K; i += blockDim.x) {
+    const int c = i / K, k = i - c * K;
+    W1s[k * C + c] = __bfloat162float(P.W1[i]);
   }
   if (warp == 1) {
     tc::tmem_alloc(tc::smem_u32(&ctl->tmem_base), kTmemCols);
@@ -301,12 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const int C = P.C, K = P.K;
-  const int C2 = 2 * C;
   const long long E = P.n_edges;
 
   if (warp == 0) {
-    // ---------------- B loader ----------------
+    // ---------------- W2 tile loader ----------------
     if (lane == 0) {
       uint32_t ib = 0;
       for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
@@ -314,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
           const TcPass& ps = P.pass[p];
           const uint32_t bytes = (uint32_t)ps.n * 128u;
           for (int j = 0; j < ps.nk; ++j, ++ib) {
-            int sb = ib % kSB;
+            const int sb = ib % kSB;
             if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kSB) & 1) ^ 1, P.status, abort, 64)) break;
             tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->b_full[sb]), bytes);
             tc::bulk_g2s(B_u32 + sb * kBStage, P.wprep + ps.boff + (long long)j * bytes, bytes,
@@ -322,10 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
           }
         }
       }
-      // drain: the newest phase of each stage must have landed before the CTA exits
+      // the newest phase of each stage must have landed before the CTA exits
       for (uint32_t k = (ib > (uint32_t)kSB ? ib - kSB : 0); k < ib; ++k) {
-        uint32_t bar = tc::smem_u32(&ctl->b_full[k % kSB]);
-        uint64_t t0 = tc::globaltimer();
+        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kSB]);
+        const uint64_t t0 = tc::globaltimer();
         while (!tc::mbar_try_wait(bar, (k / kSB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
         }
       }
@@ -333,238 +231,101 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t ia = 0, ib = 0, ip = 0, it = 0;
+      uint32_t ib = 0, ip = 0, it = 0;
       for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-        bool hid_waited = false;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full), it & 1, P.status, abort, 32)) break;
         for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
           const TcPass& ps = P.pass[p];
-          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty), (ip & 1) ^ 1, P.status, abort, 32)) break;
-          if (ps.kind == 0 && !hid_waited) {
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full), it & 1, P.status, abort, 32)) break;
-            hid_waited = true;
-          }
+          const int buf = ip & 1;
+          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty[buf]), ((ip >> 1) & 1) ^ 1, P.status, abort)) break;
           tc::tc_fence_after();
-          if (ps.kind == 1 && ps.block > 0) {
-            // y+ += x+ W1^T - x- W2^T ; y- += x+ W2^T + x- W1^T, one K block of 64 per step
-            const int np = ps.np;
-            for (int kb = 0; kb < ps.nk; ++kb, ++ib, ia += 2) {
-              const int sb = ib % kSB, sp = ia % kSA, sm = (ia + 1) % kSA;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sp]), (ia / kSA) & 1, P.status, abort, 32)) break;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sm]), ((ia + 1) / kSA) & 1, P.status, abort, 32)) break;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort, 32)) break;
-              tc::tc_fence_after();
-              const uint32_t idn = tc::idesc_f16(128, np), idneg = tc::idesc_f16(128, np, true);
+          for (int j = 0; j < ps.nk; ++j, ++ib) {
+            const int sb = ib % kSB;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
+            tc::tc_fence_after();
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ap = tc::sw128_desc(A_u32 + sp * kAStage + ks * 32);
-                const uint64_t am = tc::sw128_desc(A_u32 + sm * kAStage + ks * 32);
-                const uint64_t b1 = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
-                const uint64_t b2 = tc::sw128_desc(B_u32 + sb * kBStage + np * 128 + ks * 32);
-                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                tc::mma_bf16(tmem, ap, b1, idn, acc);
-                tc::mma_bf16(tmem, am, b2, idneg, 1u);
-                tc::mma_bf16(tmem + np, ap, b2, idn, acc);
-                tc::mma_bf16(tmem + np, am, b1, idn, 1u);
-              }
-              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sp]));
-              tc::mma_commit(tc::smem_u32(&ctl->a_empty[sm]));
-              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = tc::sw128_desc(H_u32 + j * kAStage + ks * 32);
+              const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
+              tc::mma_bf16(tmem + buf * 256, ad, bd, tc::idesc_f16(128, ps.n), (j > 0 || ks > 0) ? 1u : 0u);
             }
-          } else {
-            for (int j = 0; j < ps.nk; ++j, ++ib) {
-              const int sb = ib % kSB;
-              int sa = 0;
-              uint32_t a_base;
-              if (ps.kind == 0) {
-                a_base = H_u32 + j * kAStage;           // hidden layer, resident for the whole tile
-              } else {
-                sa = ia % kSA;
-                if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sa]), (ia / kSA) & 1, P.status, abort, 32)) break;
-                a_base = A_u32 + sa * kAStage;
-              }
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort, 32)) break;
-              tc::tc_fence_after();
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                uint64_t ad = tc::sw128_desc(a_base + ks * 32);
-                for (int n0 = 0; n0 < ps.n; n0 += 256) {
-                  int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
-                  uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + n0 * 128 + ks * 32);
-                  tc::mma_bf16(tmem + n0, ad, bd, tc::idesc_f16(128, ns), (j > 0 || ks > 0) ? 1u : 0u);
-                }
-              }
-              if (ps.kind != 0) {
-                tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
-                ++ia;
-              }
-              tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
-            }
+            tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
           }
-          if (ps.kind == 0 && ps.last_of_kind) tc::mma_commit(tc::smem_u32(&ctl->hid_empty));
-          tc::mma_commit(tc::smem_u32(&ctl->acc_full));
+          tc::mma_commit(tc::smem_u32(&ctl->acc_full[buf]));
         }
+        tc::mma_commit(tc::smem_u32(&ctl->hid_empty));
       }
       // every issued MMA must finish before TMEM is released
       tc::mma_commit(tc::smem_u32(&ctl->mma_done));
-      uint64_t t0 = tc::globaltimer();
+      const uint64_t t0 = tc::globaltimer();
       while (!tc::mbar_try_wait(tc::smem_u32(&ctl->mma_done), 0) && tc::globaltimer() - t0 < 2000000000ull) {
       }
     }
     __syncwarp();
   } else if (warp >= 2 && warp < 2 + kPW) {
-    // ---------------- A producers ----------------
-    // Coalesced mapping: the 8 lanes of a group own the eight 16-byte chunks (8 fp16
-    // channels each) of one 128-byte row slice, a warp covers 4 rows per step, and each
-    // thread walks 4 rows (rb, rb+32, rb+64, rb+96).  Every warp-wide load then touches
-    // 4 cache lines instead of 32, and a row's Wigner coefficients are broadcasts.
+    // ---------------- hidden layer ----------------
     const int pidx = (warp - 2) * 32 + lane;
-    const int q = pidx & 7;                    // 16-byte chunk within a 64-channel slice
+    const int q = pidx & 7;                    // 16-byte piece (8 channels) of a 64-channel slice
     const int rb = pidx >> 3;                  // 0..31
-    uint32_t ia = 0, it = 0;
+    const float mu_step = P.rcut / (float)(K - 1);
+    const float inv2s2 = 1.0f / (2.0f * mu_step * mu_step);
+    float b1v[2][8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b1v[j][i] = __bfloat162float(P.b1[j * 64 + q * 8 + i]);
+    uint32_t it = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-      int srcs[4], dsts[4];
-      float dists[4];
-      bool valids[4];
-      const float* Dr[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const long long e = (long long)t * 128 + rb + 32 * u;
-        valids[u] = e < E;
-        int sv = 0, dv = 0;
-        float di = 0.f;
-        if (valids[u]) {
-          sv = P.src[e];
-          int lo = 0, hi = P.n_atoms;
-          while (hi - lo > 1) {
-            int mid = (lo + hi) >> 1;
-            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
-          }
-          dv = lo;
-          if (sv < 0 || sv >= P.n_atoms) {
-            egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
-            sv = dv;
-          }
-          di = P.dist[e];
-        }
-        srcs[u] = sv;
-        dsts[u] = dv;
-        dists[u] = di;
-        Dr[u] = P.wig + (valids[u] ? e : 0) * (long long)P.wfl;
-      }
-      // radial hidden layer SiLU(W1 rho(|r_e|) + b1), once per tile, into Hbuf
       if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty), (it & 1) ^ 1, P.status, abort, 64)) break;
-      {
-        const float mu_step = P.rcut / (float)(K - 1);
-        const float inv2s2 = 1.0f / (2.0f * mu_step * mu_step);
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int r = rb + 32 * u;
+        const long long e = (long long)t * 128 + r;
+        float v[2][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = rb + 32 * u;
-          for (int j = 0; j < C / 64; ++j) {
-            const int c0 = j * 64 + q * 8;
-            float v[8];
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.f;
-            if (valids[u]) {
+          for (int i = 0; i < 8; ++i) v[j][i] = 0.f;
+        if (e < E) {
+          const float di = P.dist[e];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(P.b1[c0 + i]);
-              for (int k = 0; k < K; ++k) {
-                const float dd = dists[u] - k * mu_step;
-                const float rho = __expf(-dd * dd * inv2s2);
+          for (int j = 0; j < 2; ++j)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] += __bfloat162float(P.W1[(c0 + i) * K + k]) * rho;
-              }
+            for (int i = 0; i < 8; ++i) v[j][i] = b1v[j][i];
+          for (int k = 0; k < K; ++k) {
+            const float dd = di - k * mu_step;
+            const float rho = __expf(-dd * dd * inv2s2);
+            const float4* w = reinterpret_cast<const float4*>(W1s + k * C + q * 8);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = v[i] / (1.0f + __expf(-v[i]));
+            for (int j = 0; j < 2; ++j) {
+              const float4 w0 = w[j * 16], w1 = w[j * 16 + 1];
+              v[j][0] += w0.x * rho;
+              v[j][1] += w0.y * rho;
+              v[j][2] += w0.z * rho;
+              v[j][3] += w0.w * rho;
+              v[j][4] += w1.x * rho;
+              v[j][5] += w1.y * rho;
+              v[j][6] += w1.z * rho;
+              v[j][7] += w1.w * rho;
             }
-            uint4 w;
-            w.x = pack2h(v[0], v[1]);
-            w.y = pack2h(v[2], v[3]);
-            w.z = pack2h(v[4], v[5]);
-            w.w = pack2h(v[6], v[7]);
-            *reinterpret_cast<uint4*>(Hbuf + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
           }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[j][i] = v[j][i] / (1.0f + __expf(-v[j][i]));
         }
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(tc::smem_u32(&ctl->hid_full));
-      }
-      bool gate_waited = false;
-      for (int p = 0; p < P.npass && !*abort; ++p) {
-        const TcPass& ps = P.pass[p];
-        if (ps.kind == 0) continue;
-        if (!gate_waited) {
-          if (!tc::mbar_wait(tc::smem_u32(&ctl->gate_ready), it & 1, P.status, abort, 64)) break;
-          gate_waited = true;
-        }
-        const int b = ps.block;
-        const bool pair = b > 0;
-        const int nchunk = pair ? ps.nk : ps.nk;   // K blocks (pairs) or chunks
-        for (int j = 0; j < nchunk; ++j) {
-          const int sa0 = ia % kSA, sa1 = (ia + 1) % kSA;
-          if (!tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa0]), ((ia / kSA) & 1) ^ 1, P.status, abort, 32)) break;
-          if (pair &&
-              !tc::mbar_wait(tc::smem_u32(&ctl->a_empty[sa1]), (((ia + 1) / kSA) & 1) ^ 1, P.status, abort, 32))
-            break;
-          const int l = b + j / (C2 / 64), c2b = j % (C2 / 64);
-          const int dl = 2 * l + 1, ml = l < P.mmax ? l : P.mmax;
-          const int rp = ml + b, rm = ml - b;      // kept rows m = +b and m = -b (b = 0: the same)
-          const int cs = c2b * 64;
-          const int coff = (cs < C ? cs : cs - C) + q * 8;
-          __half2 ap[4][4], am[4][4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) ap[u][i] = am[u][i] = __float2half2_rn(0.f);
-          for (int mp = 0; mp < dl; ++mp) {
-            uint4 zq[4];
-            __half2 cp[4], cm[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int node = cs < C ? srcs[u] : dsts[u];
-              zq[u] = valids[u] ? __ldg(reinterpret_cast<const uint4*>(
-                                      P.node_h + ((long long)node * P.L2 + l * l + mp) * C + coff))
-                                : make_uint4(0, 0, 0, 0);
-              const float* Dl = Dr[u] + P.woff[l];
-              cp[u] = __float2half2_rn(valids[u] ? __ldg(Dl + rp * dl + mp) : 0.f);
-              cm[u] = __float2half2_rn(valids[u] && pair ? __ldg(Dl + rm * dl + mp) : 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const __half2* h = reinterpret_cast<const __half2*>(&zq[u]);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                ap[u][i] = __hfma2(cp[u], h[i], ap[u][i]);
-                if (pair) am[u][i] = __hfma2(cm[u], h[i], am[u][i]);
-              }
-            }
-          }
-          uint8_t* tp = Abuf + sa0 * kAStage;
-          uint8_t* tm = Abuf + sa1 * kAStage;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int r = rb + 32 * u;
-            const uint4 gw = *reinterpret_cast<const uint4*>(P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols +
-                                                             l * C2 + cs + q * 8);
-            const __half2* g = reinterpret_cast<const __half2*>(&gw);
-            uint4 wp, wm;
-            uint32_t* pp = reinterpret_cast<uint32_t*>(&wp);
-            uint32_t* pm = reinterpret_cast<uint32_t*>(&wm);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const __half2 xp = __hmul2(ap[u][i], g[i]);
-              const __half2 xm = __hmul2(am[u][i], g[i]);
-              pp[i] = *reinterpret_cast<const uint32_t*>(&xp);
-              pm[i] = *reinterpret_cast<const uint32_t*>(&xm);
-            }
-            const int off = r * 128 + ((q ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(tp + off) = wp;
-            if (pair) *reinterpret_cast<uint4*>(tm + off) = wm;
-          }
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa0]));
-          if (pair) tc::mbar_arrive(tc::smem_u32(&ctl->a_full[sa1]));
-          ia += pair ? 2 : 1;
+        for (int j = 0; j < 2; ++j) {
+          uint4 w;
+          w.x = pack2h(v[j][0], v[j][1]);
+          w.y = pack2h(v[j][2], v[j][3]);
+          w.z = pack2h(v[j][4], v[j][5]);
+          w.w = pack2h(v[j][6], v[j][7]);
+          *reinterpret_cast<uint4*>(Hbuf + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
         }
       }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(tc::smem_u32(&ctl->hid_full));
     }
   } else {
     // ---------------- epilogue: thread = TMEM lane = edge ----------------
@@ -574,23 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1) so2_tc_kernel(const __grid_consta
     uint32_t ip = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
       const long long e = (long long)t * 128 + r;
-      const bool valid = e < E;
-      __half* gsc = P.gates ? P.gates + ((long long)(t - P.t_begin) * 128 + r) * P.gcols
-                            : P.gate_scratch + ((long long)blockIdx.x * 128 + r) * P.gcols;
+      __half* gsc = P.gates + ((long long)(t - P.t_begin) * 128 + r) * P.gcols;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
-        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full), ip & 1, P.status, abort, 256)) break;
+        const int buf = ip & 1;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), (ip >> 1) & 1, P.status, abort, 64)) break;
         tc::tc_fence_after();
         for (int g = 0; g < ps.n; g += 32) {
           uint32_t ra[32];
-          tc::tmem_ld32_issue(tl + g, ra);
+          tc::tmem_ld32_issue(tl + buf * 256 + g, ra);
           tc::tmem_ld_wait(ra);
-          epi_store(P, ps, gsc, e, valid, g, ra);
+          epi_store(P, ps, gsc, e, true, g, ra);
         }
         tc::tc_fence_before();
-        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty));
-        if (ps.kind == 0 && ps.last_of_kind) tc::mbar_arrive(tc::smem_u32(&ctl->gate_ready));
-
+        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
       }
     }
   }
@@ -1323,7 +1081,9 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
 
 }  // namespace
 
-size_t so2_tc_smem_bytes() { return kSA * kAStage + kSB * kBStage + kHStage + sizeof(SmemCtl) + 1024; }
+size_t gate_smem_bytes(int K, int C) {
+  return kSB * kBStage + kHStage + sizeof(float) * (size_t)K * C + sizeof(GateCtl) + 1024;
+}
 
 // bf16 -> fp16 copy of the node table (exact for the embeddings' range), 8 values per thread.
 __global__ void to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half* __restrict__ out, long long n8) {
@@ -1388,9 +1148,9 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
   Pg.npass = ng;
   Ps.npass = P.npass - ng;
   for (int i = 0; i < Ps.npass; ++i) Ps.pass[i] = P.pass[ng + i];
-  const size_t sm_g = so2_tc_smem_bytes();
+  const size_t sm_g = gate_smem_bytes(P.K, P.C);
   const size_t sm_s = kGA * kAStage + kSB * kBStage + sizeof(GemmCtl) + 1024;
-  if ((err = cudaFuncSetAttribute(so2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) !=
+  if ((err = cudaFuncSetAttribute(gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) !=
       cudaSuccess)
     return err;
   if ((err = cudaFuncSetAttribute(so2_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_s)) !=
@@ -1403,7 +1163,7 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
     const int grid = P.grid < nt ? P.grid : nt;
     Pg.t_begin = Ps.t_begin = tb;
     Pg.t_end = Ps.t_end = te;
-    so2_tc_kernel<<<grid, kThreads, sm_g, st>>>(Pg);
+    gate_kernel<<<grid, kThreads, sm_g, st>>>(Pg);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if ((err = launch_rotate_any(Ps, nt, st)) != cudaSuccess) return err;
     so2_gemm_kernel<<<grid, kGThreads, sm_s, st>>>(Ps);

@@ -39,7 +39,6 @@ struct TcParams {
   const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
   const uint8_t* wprep;
   long long wprep_bytes;
-  __half* gate_scratch;          // [grid][128][gcols] radial gates, fp16
   uint8_t* Y;                    // [n_edges][y_row_bytes]
   float* logits;                 // [n_edges][H]
   float* Af;                     // attention matrix A[H][L*C] in fp32 (workspace copy)
@@ -90,7 +89,7 @@ struct HeadUPtrs {
   const __nv_bfloat16* U[8];
 };
 
-size_t so2_tc_smem_bytes();
+size_t gate_smem_bytes(int K, int C);
 cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st);
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
                            float* blocks, cudaStream_t st);

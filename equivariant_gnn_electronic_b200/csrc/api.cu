@@ -101,8 +101,9 @@ bool tc_eligible(const egnn_layer_desc* d) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Pass list: radial-gate passes, then the SO(2) blocks |m| = 0..mmax, each block's
-// output rows split into accumulators of at most 512 TMEM columns.  With `mult`
+// Pass list: radial-gate passes (256 columns each), then the SO(2) blocks
+// |m| = 0..mmax, each block's output rows split into accumulators of at most
+// kTcAccCols TMEM columns.  With `mult`
 // (head, label mode) the output rows of block b are the labels (l >= b, k < mult_l)
 // instead of the channels (l >= b, c < C).  Returns false if the plan needs more
 // passes than TcParams holds.
@@ -114,9 +115,9 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
   long long boff = 0;
   int roff = 0;
   auto add = [&](int kind, int block, int ntot, int nk) -> bool {
-    const int step = kind == 0 ? 256 : 512;   // gate passes alternate two 256-column accumulators
+    const int step = kind == 0 ? 256 : kTcAccCols;   // gate passes alternate two 256-column accumulators
     for (int off = 0; off < ntot; off += step) {
-      if (P.npass >= 16) return false;
+      if (P.npass >= 32) return false;
       TcPass& q = P.pass[P.npass++];
       q.kind = kind;
       q.block = block;
@@ -159,12 +160,12 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
     const int kblocks = (L - b) * 2 * C / 64;
     P.ybase[b] = ycol;
     ycol += 2 * (L - b) * C;
-    for (int o0 = 0; o0 < nC; o0 += 256) {
-      if (P.npass >= 16) return false;
+    for (int o0 = 0; o0 < nC; o0 += kTcPairRows) {
+      if (P.npass >= 32) return false;
       TcPass& q = P.pass[P.npass++];
       q.kind = 1;
       q.block = b;
-      q.np = nC - o0 < 256 ? nC - o0 : 256;
+      q.np = nC - o0 < kTcPairRows ? nC - o0 : kTcPairRows;
       if (label) q.np = (q.np + 15) & ~15;
       q.n = 2 * q.np;
       q.n_off = o0;

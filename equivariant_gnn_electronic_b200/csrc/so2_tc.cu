@@ -22,13 +22,14 @@
 //                 the CUDA cores), fp16 per edge;
 //   rotate        x_e = g_e * (D^l(R_e) [n_s || n_d]) for the kept rows |m| <= mmax,
 //                 written as ready-made A tiles;
-//   so2_gemm      D[128 x N <= 512] = A[128 x K] B[N x K]^T per pass in TMEM, with
-//                 B = W0 (|m| = 0) or [W_b1 ; W_b2] read by four MMAs, one with the
-//                 negate-B bit, per K block (|m| = b > 0); the epilogue writes y_e
-//                 (y0 in fp32, |m| > 0 in bf16) or, for the head, edge-frame labels.
-//   Then logits (attention logits from SiLU(y0)) and agg (one CTA per destination
-//   atom: softmax over its incoming edges, rotate back with the kept rows of D^l,
-//   weighted sum, residual; no atomics).
+//   so2_gemm      D[128 x N <= 256] = A[128 x K] B[N x K]^T per pass in one of two
+//                 alternating TMEM accumulators, with B = W0 (|m| = 0) or
+//                 [W_b1 ; W_b2] read by four MMAs, one with the negate-B bit, per K
+//                 block (|m| = b > 0); the epilogue writes y_e (y0 in fp32, |m| > 0
+//                 in bf16) and the attention logits A SiLU(y0_e) + bA, or, for the
+//                 head, edge-frame labels.
+//   Then agg (one CTA per destination atom: softmax over its incoming edges, rotate
+//   back with the kept rows of D^l, weighted sum, residual; no atomics).
 #include <math.h>
 
 #include "common.cuh"
@@ -38,9 +39,9 @@
 
 namespace {
 
-constexpr int kSB = 2;                 // B stages (<= 512 x 64 fp16 = 64 KB each)
+constexpr int kSB = 2;                 // gate kernel B stages
 constexpr int kAStage = 128 * 128;     // one 128 x 64 fp16 A tile (16 KB)
-constexpr int kBStage = 512 * 128;
+constexpr int kBStage = 256 * 128;     // one <= 256 x 64 fp16 B tile (32 KB)
 constexpr int kTmemCols = 512;
 constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = C = 128: two A tiles
 constexpr int kPW = 8;                 // gate kernel: warps computing the hidden layer
@@ -49,7 +50,7 @@ constexpr int kThreads = (2 + kPW + 4) * 32;   // 0 loader, 1 MMA, hidden layer,
 
 struct GateCtl {
   uint64_t b_full[kSB], b_empty[kSB], acc_full[2], acc_empty[2];
-  uint64_t hid_full, hid_empty, mma_done;
+  uint64_t hid_full[2], hid_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -73,84 +74,62 @@ __device__ __forceinline__ uint32_t pack2h(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Epilogue store of one 32-column group of a pass (thread = edge row): gate passes
-// add b2 and keep fp16 gates in the CTA's scratch; SO(2) passes write y (y0 in fp32,
-// the |m| > 0 blocks in bf16).
-__device__ __forceinline__ void epi_store(const TcParams& P, const TcPass& ps, __half* gsc, long long e, bool valid,
-                                          int g, const uint32_t* ru) {
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ru[i]);
+// Epilogue store of one 32-column group of a pass, cooperative over a warp that owns
+// 32 consecutive TMEM lanes (rows).  Each thread stages its row's 32 values in the
+// warp's shared-memory tile (row stride 36 floats: 16-byte aligned, conflict-free for
+// both the row-wise writes and the column-wise reads); the warp then writes 4 rows
+// per instruction, each row's 32 columns contiguous, so every store covers whole
+// 128-byte (fp32) or 64-byte (16-bit) segments instead of 32 scattered pieces.
+// Gate passes add b2 and write fp16 gates; SO(2) passes write y (y0 in fp32, the
+// |m| > 0 blocks in bf16) or, in label mode, the fp32 label record.
+constexpr int kStageFloats = 32 * 36;   // per warp
+__device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& ps, float* st, long long e0,
+                                               long long grow0, int g, const uint32_t* ru) {
+  const int lane = threadIdx.x & 31;
   int col = ps.n_off + g;
-  if (ps.kind == 1 && ps.block > 0 && g >= ps.np) col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
-  if (ps.kind == 0) {
+  if (ps.kind == 1 && ps.block > 0 && !P.label_mode && g >= ps.np)
+    col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
+  float4* srow = reinterpret_cast<float4*>(st + lane * 36);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] += __bfloat162float(P.b2[col + i]);
-    uint4* dst = reinterpret_cast<uint4*>(gsc + col);
+  for (int q = 0; q < 8; ++q) {
+    float4 x = make_float4(__uint_as_float(ru[4 * q]), __uint_as_float(ru[4 * q + 1]),
+                           __uint_as_float(ru[4 * q + 2]), __uint_as_float(ru[4 * q + 3]));
+    if (ps.kind == 0) {
+      x.x += __bfloat162float(P.b2[col + 4 * q]);
+      x.y += __bfloat162float(P.b2[col + 4 * q + 1]);
+      x.z += __bfloat162float(P.b2[col + 4 * q + 2]);
+      x.w += __bfloat162float(P.b2[col + 4 * q + 3]);
+    }
+    srow[q] = x;
+  }
+  __syncwarp();
+  const int c4 = (lane & 7) * 4, rs = lane >> 3;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(pack2h(v[8 * q], v[8 * q + 1]), pack2h(v[8 * q + 2], v[8 * q + 3]),
-                          pack2h(v[8 * q + 4], v[8 * q + 5]), pack2h(v[8 * q + 6], v[8 * q + 7]));
-  } else if (valid) {
-    uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
-    if (P.label_mode) {
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + ps.roff + g);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = make_uint4(ru[4 * q], ru[4 * q + 1], ru[4 * q + 2], ru[4 * q + 3]);
-    } else if (ps.block == 0) {
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(yrow) + col);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = make_uint4(ru[4 * q], ru[4 * q + 1], ru[4 * q + 2], ru[4 * q + 3]);
+  for (int r0 = 0; r0 < 32; r0 += 4) {
+    const int rr = r0 + rs;
+    const float4 x = *reinterpret_cast<const float4*>(st + rr * 36 + c4);
+    if (ps.kind == 0) {
+      __half* dst = P.gates + (grow0 + rr) * P.gcols + col + c4;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack2h(x.x, x.y), pack2h(x.z, x.w));
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) +
-                                            (P.ybase[ps.block] - P.ybase[1]) + col);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        dst[q] = make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
-                            pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
+      const long long e = e0 + rr;
+      if (e < P.n_edges) {
+        uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
+        if (P.label_mode) {
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + ps.roff + g + c4) = x;
+        } else if (ps.block == 0) {
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + col + c4) = x;
+        } else {
+          __nv_bfloat16* dst =
+              reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) + (P.ybase[ps.block] - P.ybase[1]) + col + c4;
+          *reinterpret_cast<uint2*>(dst) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+        }
+      }
     }
   }
+  __syncwarp();
 }
 
-// Attention logits a_{e,h} = A[h] . SiLU(y0_e) + bA[h], one warp per edge: lanes
-// read y0 (fp32, coalesced) and the fp32 copy of A staged in shared memory, then the
-// heads' partial sums are reduced across the warp.
-__global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcParams P) {
-  extern __shared__ float As[];                 // [H][L*C]
-  const int LC = P.L * P.C, H = P.H;
-  for (int i = threadIdx.x; i < H * LC; i += blockDim.x) As[i] = P.Af[i];
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < P.n_edges; e += nw) {
-    const float* y0 = reinterpret_cast<const float*>(P.Y + e * (long long)P.y_row_bytes);
-    float a[16];
-#pragma unroll
-    for (int h = 0; h < 16; ++h) a[h] = 0.f;
-    float yv[28];                                // LC <= 7 * 128 = 896 = 28 * 32: all loads first
-#pragma unroll
-    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
-#pragma unroll
-    for (int k = 0; k < 28; ++k) {
-      const int j = lane + 32 * k;
-      if (j < LC) {
-        const float sv = yv[k] / (1.0f + __expf(-yv[k]));
-#pragma unroll
-        for (int h = 0; h < 16; ++h)
-          if (h < H) a[h] += As[h * LC + j] * sv;
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < 16; ++h) {
-      if (h < H) {
-        float x = a[h];
-#pragma unroll
-        for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        if (lane == 0) P.logits[e * H + h] = x + __bfloat162float(P.bA[h]);
-      }
-    }
-  }
-}
 
 // Radial gate GEMM, persistent over the tiles of a range: per 128-edge tile the
 // hidden layer h = SiLU(W1 rho(|r_e|) + b1) (K Gaussians) is computed on the CUDA
@@ -166,8 +145,9 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
   uint8_t* Hbuf = base + kSB * kBStage;
-  float* W1s = reinterpret_cast<float*>(Hbuf + kHStage);   // [K][C] fp32
-  GateCtl* ctl = reinterpret_cast<GateCtl*>(W1s + P.K * P.C);
+  float* W1s = reinterpret_cast<float*>(Hbuf + 2 * kHStage);   // [K][C] fp32 (after two hidden buffers)
+  float* Stg = W1s + P.K * P.C;                              // epilogue staging, 4 warps
+  GateCtl* ctl = reinterpret_cast<GateCtl*>(Stg + 4 * kStageFloats);
   const uint32_t B_u32 = base_u32;
   const uint32_t H_u32 = base_u32 + kSB * kBStage;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,8 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
       tc::mbar_init(tc::smem_u32(&ctl->acc_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->acc_empty[i]), 128);
     }
-    tc::mbar_init(tc::smem_u32(&ctl->hid_full), kProducers);
-    tc::mbar_init(tc::smem_u32(&ctl->hid_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->hid_full[i]), kProducers);
+      tc::mbar_init(tc::smem_u32(&ctl->hid_empty[i]), 1);
+    }
     tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
     ctl->abort = 0;
     tc::fence_barrier_init();
@@ -233,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
     if (lane == 0) {
       uint32_t ib = 0, ip = 0, it = 0;
       for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-        if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full), it & 1, P.status, abort, 32)) break;
+        const int hb = it & 1;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full[hb]), (it >> 1) & 1, P.status, abort, 32)) break;
         for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
           const TcPass& ps = P.pass[p];
           const int buf = ip & 1;
@@ -245,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
             tc::tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = tc::sw128_desc(H_u32 + j * kAStage + ks * 32);
+              const uint64_t ad = tc::sw128_desc(H_u32 + hb * kHStage + j * kAStage + ks * 32);
               const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
               tc::mma_bf16(tmem + buf * 256, ad, bd, tc::idesc_f16(128, ps.n), (j > 0 || ks > 0) ? 1u : 0u);
             }
@@ -253,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
           }
           tc::mma_commit(tc::smem_u32(&ctl->acc_full[buf]));
         }
-        tc::mma_commit(tc::smem_u32(&ctl->hid_empty));
+        tc::mma_commit(tc::smem_u32(&ctl->hid_empty[hb]));
       }
       // every issued MMA must finish before TMEM is released
       tc::mma_commit(tc::smem_u32(&ctl->mma_done));
@@ -276,7 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
       for (int i = 0; i < 8; ++i) b1v[j][i] = __bfloat162float(P.b1[j * 64 + q * 8 + i]);
     uint32_t it = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-      if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty), (it & 1) ^ 1, P.status, abort, 64)) break;
+      const int hb = it & 1;
+      uint8_t* Hb = Hbuf + hb * kHStage;
+      if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty[hb]), ((it >> 1) & 1) ^ 1, P.status, abort, 64)) break;
 #pragma unroll 1
       for (int u = 0; u < 4; ++u) {
         const int r = rb + 32 * u;
@@ -321,31 +306,40 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
           w.y = pack2h(v[j][2], v[j][3]);
           w.z = pack2h(v[j][4], v[j][5]);
           w.w = pack2h(v[j][6], v[j][7]);
-          *reinterpret_cast<uint4*>(Hbuf + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
+          *reinterpret_cast<uint4*>(Hb + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
         }
       }
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(tc::smem_u32(&ctl->hid_full));
+      tc::mbar_arrive(tc::smem_u32(&ctl->hid_full[hb]));
     }
   } else {
     // ---------------- epilogue: thread = TMEM lane = edge ----------------
     const int sub = warp & 3;
-    const int r = sub * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
+    float* st = Stg + sub * kStageFloats;
     uint32_t ip = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
-      const long long e = (long long)t * 128 + r;
-      __half* gsc = P.gates + ((long long)(t - P.t_begin) * 128 + r) * P.gcols;
+      const long long grow0 = (long long)(t - P.t_begin) * 128 + sub * 32;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
         const int buf = ip & 1;
         if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), (ip >> 1) & 1, P.status, abort, 64)) break;
         tc::tc_fence_after();
-        for (int g = 0; g < ps.n; g += 32) {
-          uint32_t ra[32];
-          tc::tmem_ld32_issue(tl + buf * 256 + g, ra);
-          tc::tmem_ld_wait(ra);
-          epi_store(P, ps, gsc, e, true, g, ra);
+        // the TMEM load of the next 32 columns is in flight while the current ones are stored
+        const uint32_t tb = tl + buf * 256;
+        uint32_t ra[32], rb[32];
+        tc::tmem_ld32_issue(tb, ra);
+        tc::tmem_ld_wait(ra);
+        for (int g = 0; g < ps.n; g += 64) {
+          const bool h1 = g + 32 < ps.n, h2 = g + 64 < ps.n;
+          if (h1) tc::tmem_ld32_issue(tb + g + 32, rb);
+          epi_store_warp(P, ps, st, 0, grow0, g, ra);
+          if (h1) {
+            tc::tmem_ld_wait(rb);
+            if (h2) tc::tmem_ld32_issue(tb + g + 64, ra);
+            epi_store_warp(P, ps, st, 0, grow0, g + 32, rb);
+            if (h2) tc::tmem_ld_wait(ra);
+          }
         }
         tc::tc_fence_before();
         tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
@@ -765,10 +759,11 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
     const float* Re = Rs + e * nrec;
     float h = De[ml * dl] * Re[s_hroff[0] + s_lb[0][Lq] + k];
     for (int b = 1; b <= ml; ++b) {
-      const int r = s_lb[b][Lq] + k, qq = r >> 8, w = r & 255;
-      const int rest = s_hnr[b] - 256 * qq;
-      const int npq = rest >= 256 ? 256 : ((rest + 15) & ~15);
-      const int base = s_hroff[b] + 512 * qq + w;
+      // pass qq of block b holds label rows [R qq, R qq + npq) of s+ then of s-, R = kTcPairRows
+      const int r = s_lb[b][Lq] + k, qq = r / kTcPairRows, w = r - qq * kTcPairRows;
+      const int rest = s_hnr[b] - kTcPairRows * qq;
+      const int npq = rest >= kTcPairRows ? kTcPairRows : ((rest + 15) & ~15);
+      const int base = s_hroff[b] + 2 * kTcPairRows * qq + w;
       h += De[(ml + b) * dl] * Re[base] + De[(ml - b) * dl] * Re[base + npq];
     }
     Ls[e * nlab + q0] = h;
@@ -792,6 +787,46 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
   }
 }
 
+
+// Attention logits a_{e,h} = A[h] . SiLU(y0_e) + bA[h], one warp per edge: lanes
+// read y0 (fp32, coalesced) and the fp32 copy of A staged in shared memory, then the
+// heads' partial sums are reduced across the warp.
+__global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ float As[];                 // [H][L*C]
+  const int LC = P.L * P.C, H = P.H;
+  for (int i = threadIdx.x; i < H * LC; i += blockDim.x) As[i] = P.Af[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < P.n_edges; e += nw) {
+    const float* y0 = reinterpret_cast<const float*>(P.Y + e * (long long)P.y_row_bytes);
+    float a[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) a[h] = 0.f;
+    float yv[28];                                // LC <= 7 * 128 = 896 = 28 * 32: all loads first
+#pragma unroll
+    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 28; ++k) {
+      const int j = lane + 32 * k;
+      if (j < LC) {
+        const float sv = yv[k] / (1.0f + __expf(-yv[k]));
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+          if (h < H) a[h] += As[h * LC + j] * sv;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+      if (h < H) {
+        float x = a[h];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (lane == 0) P.logits[e * H + h] = x + __bfloat162float(P.bA[h]);
+      }
+    }
+  }
+}
 
 // ---------------- rotate + gate: the A operands of the SO(2) GEMM ----------------
 // One CTA per 128-edge tile.  For every edge and degree l the kept rows of the edge
@@ -898,12 +933,15 @@ __global__ void __launch_bounds__(256) rotate_kernel(const __grid_constant__ TcP
 // Persistent over the tiles of a range.  Warp 0 bulk-copies the prepared A tiles of
 // the rotate kernel and the weight tiles, warp 1 issues the MMAs (one thread) and
 // owns TMEM, warps 2-5 drain each pass's accumulator (thread = TMEM lane = edge).
-constexpr int kGA = 6;                 // A stages (16 KB each)
+constexpr int kNBuf = kTcAccCols == 256 ? 2 : 1;    // TMEM accumulators
+constexpr int kGA = kNBuf == 2 ? 6 : 4;              // A stages (16 KB each)
+constexpr int kGB = kNBuf == 2 ? 3 : 2;              // B stages
+constexpr int kGBStage = kTcAccCols * 128;           // one <= kTcAccCols x 64 fp16 B tile
 constexpr int kGThreads = 6 * 32;
 
 struct GemmCtl {
-  uint64_t a_full[kGA], a_empty[kGA], b_full[kSB], b_empty[kSB];
-  uint64_t acc_full, acc_empty, mma_done;
+  uint64_t a_full[kGA], a_empty[kGA], b_full[kGB], b_empty[kGB];
+  uint64_t acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -913,7 +951,8 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
-  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(base + kGA * kAStage + kSB * kBStage);
+  float* Stg = reinterpret_cast<float*>(base + kGA * kAStage + kGB * kGBStage);   // epilogue staging
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(Stg + 4 * kStageFloats);
   const uint32_t A_u32 = base_u32;
   const uint32_t B_u32 = base_u32 + kGA * kAStage;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -924,12 +963,14 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
       tc::mbar_init(tc::smem_u32(&ctl->a_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->a_empty[i]), 1);
     }
-    for (int i = 0; i < kSB; ++i) {
+    for (int i = 0; i < kGB; ++i) {
       tc::mbar_init(tc::smem_u32(&ctl->b_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->b_empty[i]), 1);
     }
-    tc::mbar_init(tc::smem_u32(&ctl->acc_full), 1);
-    tc::mbar_init(tc::smem_u32(&ctl->acc_empty), 128);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->acc_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->acc_empty[i]), 128);
+    }
     tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
     ctl->abort = 0;
     tc::fence_barrier_init();
@@ -954,10 +995,10 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
           const uint32_t bytes = (uint32_t)ps.n * 128u;
           const int na = ps.block > 0 ? 2 : 1;
           for (int kb = 0; kb < ps.nk && !*abort; ++kb, ++ib) {
-            const int sb = ib % kSB;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kSB) & 1) ^ 1, P.status, abort, 64)) break;
+            const int sb = ib % kGB;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kGB) & 1) ^ 1, P.status, abort, 64)) break;
             tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->b_full[sb]), bytes);
-            tc::bulk_g2s(B_u32 + sb * kBStage, P.wprep + ps.boff + (long long)kb * bytes, bytes,
+            tc::bulk_g2s(B_u32 + sb * kGBStage, P.wprep + ps.boff + (long long)kb * bytes, bytes,
                          tc::smem_u32(&ctl->b_full[sb]));
             for (int h = 0; h < na; ++h, ++ia) {
               const int sa = ia % kGA;
@@ -971,10 +1012,10 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
         }
       }
       // the newest phase of every stage must have landed before the CTA exits
-      for (uint32_t k = (ib > (uint32_t)kSB ? ib - kSB : 0); k < ib; ++k) {
-        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kSB]);
+      for (uint32_t k = (ib > (uint32_t)kGB ? ib - kGB : 0); k < ib; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kGB]);
         const uint64_t t0 = tc::globaltimer();
-        while (!tc::mbar_try_wait(bar, (k / kSB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        while (!tc::mbar_try_wait(bar, (k / kGB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
         }
       }
       for (uint32_t k = (ia > (uint32_t)kGA ? ia - kGA : 0); k < ia; ++k) {
@@ -990,15 +1031,18 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
       for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
         for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
           const TcPass& ps = P.pass[p];
-          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty), (ip & 1) ^ 1, P.status, abort, 32)) break;
+          const int buf = kNBuf == 2 ? (ip & 1) : 0;
+          const uint32_t ph = kNBuf == 2 ? (ip >> 1) & 1 : ip & 1;
+          const uint32_t acc_t = tmem + buf * 256;
+          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty[buf]), ph ^ 1, P.status, abort, 32)) break;
           tc::tc_fence_after();
           if (ps.block > 0) {
             // y+ += x+ W1^T - x- W2^T ; y- += x+ W2^T + x- W1^T, one K block of 64 per step
             const int np = ps.np;
             const uint32_t idn = tc::idesc_f16(128, np), idneg = tc::idesc_f16(128, np, true);
             for (int kb = 0; kb < ps.nk; ++kb, ++ib, ia += 2) {
-              const int sb = ib % kSB, sp = ia % kGA, sm = (ia + 1) % kGA;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
+              const int sb = ib % kGB, sp = ia % kGA, sm = (ia + 1) % kGA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kGB) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sp]), (ia / kGA) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sm]), ((ia + 1) / kGA) & 1, P.status, abort)) break;
               tc::tc_fence_after();
@@ -1006,13 +1050,13 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
               for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ap = tc::sw128_desc(A_u32 + sp * kAStage + ks * 32);
                 const uint64_t am = tc::sw128_desc(A_u32 + sm * kAStage + ks * 32);
-                const uint64_t b1 = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
-                const uint64_t b2 = tc::sw128_desc(B_u32 + sb * kBStage + np * 128 + ks * 32);
+                const uint64_t b1 = tc::sw128_desc(B_u32 + sb * kGBStage + ks * 32);
+                const uint64_t b2 = tc::sw128_desc(B_u32 + sb * kGBStage + np * 128 + ks * 32);
                 const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                tc::mma_bf16(tmem, ap, b1, idn, acc);
-                tc::mma_bf16(tmem, am, b2, idneg, 1u);
-                tc::mma_bf16(tmem + np, ap, b2, idn, acc);
-                tc::mma_bf16(tmem + np, am, b1, idn, 1u);
+                tc::mma_bf16(acc_t, ap, b1, idn, acc);
+                tc::mma_bf16(acc_t, am, b2, idneg, 1u);
+                tc::mma_bf16(acc_t + np, ap, b2, idn, acc);
+                tc::mma_bf16(acc_t + np, am, b1, idn, 1u);
               }
               tc::mma_commit(tc::smem_u32(&ctl->a_empty[sp]));
               tc::mma_commit(tc::smem_u32(&ctl->a_empty[sm]));
@@ -1020,8 +1064,8 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
             }
           } else {
             for (int kb = 0; kb < ps.nk; ++kb, ++ib, ++ia) {
-              const int sb = ib % kSB, sa = ia % kGA;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
+              const int sb = ib % kGB, sa = ia % kGA;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kGB) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->a_full[sa]), (ia / kGA) & 1, P.status, abort)) break;
               tc::tc_fence_after();
 #pragma unroll
@@ -1029,15 +1073,15 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
                 const uint64_t ad = tc::sw128_desc(A_u32 + sa * kAStage + ks * 32);
                 for (int n0 = 0; n0 < ps.n; n0 += 256) {
                   const int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
-                  const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + n0 * 128 + ks * 32);
-                  tc::mma_bf16(tmem + n0, ad, bd, tc::idesc_f16(128, ns), (kb > 0 || ks > 0) ? 1u : 0u);
+                  const uint64_t bd = tc::sw128_desc(B_u32 + sb * kGBStage + n0 * 128 + ks * 32);
+                  tc::mma_bf16(acc_t + n0, ad, bd, tc::idesc_f16(128, ns), (kb > 0 || ks > 0) ? 1u : 0u);
                 }
               }
               tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
               tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
             }
           }
-          tc::mma_commit(tc::smem_u32(&ctl->acc_full));
+          tc::mma_commit(tc::smem_u32(&ctl->acc_full[buf]));
         }
       }
       // every issued MMA must finish before TMEM is released
@@ -1052,22 +1096,57 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
+    float* st = Stg + sub * kStageFloats;
+    const int LC = P.L * P.C, H = P.H;
+    const bool logits = kTcLogitsInEpilogue && P.with_logits && !P.label_mode;
     uint32_t ip = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
       const long long e = (long long)t * 128 + r;
       const bool valid = e < E;
+      float la[16];   // attention logits of this edge, accumulated over the |m| = 0 passes
+#pragma unroll
+      for (int h = 0; h < 16; ++h) la[h] = 0.f;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
-        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full), ip & 1, P.status, abort, 128)) break;
+        const int buf = kNBuf == 2 ? (ip & 1) : 0;
+        const uint32_t ph = kNBuf == 2 ? (ip >> 1) & 1 : ip & 1;
+        const uint32_t tb = tl + buf * 256;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), ph, P.status, abort, 128)) break;
         tc::tc_fence_after();
+        const bool lg = logits && ps.block == 0;
         for (int g = 0; g < ps.n; g += 32) {
           uint32_t ra[32];
-          tc::tmem_ld32_issue(tl + g, ra);
+          tc::tmem_ld32_issue(tb + g, ra);
           tc::tmem_ld_wait(ra);
-          epi_store(P, ps, nullptr, e, valid, g, ra);
+          epi_store_warp(P, ps, st, (long long)t * 128 + sub * 32, 0, g, ra);
+          if (lg) {
+            // a_h += A[h, j] SiLU(y0_j) over this group's 32 columns j of y0
+            const float* Ag = P.Af + ps.n_off + g;
+#pragma unroll
+            for (int i4 = 0; i4 < 8; ++i4) {
+              float sv[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float y = __uint_as_float(ra[4 * i4 + c]);
+                sv[c] = y / (1.0f + __expf(-y));
+              }
+#pragma unroll
+              for (int h = 0; h < 16; ++h) {
+                if (h < H) {
+                  const float4 a = __ldg(reinterpret_cast<const float4*>(Ag + h * LC) + i4);
+                  la[h] += a.x * sv[0] + a.y * sv[1] + a.z * sv[2] + a.w * sv[3];
+                }
+              }
+            }
+          }
         }
         tc::tc_fence_before();
-        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty));
+        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
+        if (lg && ps.last_of_kind && valid) {
+#pragma unroll
+          for (int h = 0; h < 16; ++h)
+            if (h < H) P.logits[e * H + h] = la[h] + __bfloat162float(P.bA[h]);
+        }
       }
     }
   }
@@ -1082,7 +1161,7 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
 }  // namespace
 
 size_t gate_smem_bytes(int K, int C) {
-  return kSB * kBStage + kHStage + sizeof(float) * (size_t)K * C + sizeof(GateCtl) + 1024;
+  return kSB * kBStage + 2 * kHStage + sizeof(float) * ((size_t)K * C + 4 * kStageFloats) + sizeof(GateCtl) + 1024;
 }
 
 // bf16 -> fp16 copy of the node table (exact for the embeddings' range), 8 values per thread.
@@ -1149,7 +1228,7 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
   Ps.npass = P.npass - ng;
   for (int i = 0; i < Ps.npass; ++i) Ps.pass[i] = P.pass[ng + i];
   const size_t sm_g = gate_smem_bytes(P.K, P.C);
-  const size_t sm_s = kGA * kAStage + kSB * kBStage + sizeof(GemmCtl) + 1024;
+  const size_t sm_s = kGA * kAStage + kGB * kGBStage + sizeof(float) * 4 * kStageFloats + sizeof(GemmCtl) + 1024;
   if ((err = cudaFuncSetAttribute(gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) !=
       cudaSuccess)
     return err;
@@ -1223,11 +1302,13 @@ cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTabl
 cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st) {
   cudaError_t err = launch_tc_gemm(P, W, st);
   if (err != cudaSuccess) return err;
-  if (P.n_edges > 0) {
+  if (!kTcLogitsInEpilogue && P.n_edges > 0) {
     const size_t sm = sizeof(float) * (size_t)P.H * P.L * P.C;
     err = cudaFuncSetAttribute(logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (err != cudaSuccess) return err;
-    logits_kernel<<<2 * P.grid, 256, sm, st>>>(P);
+    int nb = 2;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, logits_kernel, 256, sm);
+    logits_kernel<<<(nb > 0 ? nb : 1) * P.grid, 256, sm, st>>>(P);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

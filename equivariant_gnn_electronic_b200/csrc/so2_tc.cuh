@@ -5,14 +5,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-// One GEMM pass over a 128-edge tile: D[128 x n] = A[128 x 64*nk] B[n x 64*nk]^T.  For a
-// block with |m| = b > 0 the pass covers output rows [n_off, n_off + np) of both y+ and
-// y- (n = 2 np) and B holds only the rows of W_b1 and W_b2 (the sign comes from the
-// instruction's negate-B bit), so each weight is streamed once.
+// One GEMM pass over a 128-edge tile: D[128 x n] = A[128 x 64*nk] B[n x 64*nk]^T, n <= 256
+// so that two accumulators alternate in TMEM.  For a block with |m| = b > 0 the pass
+// covers output rows [n_off, n_off + np) of both y+ and y- (n = 2 np) and B holds only
+// the rows of W_b1 and W_b2 (the sign comes from the instruction's negate-B bit).
 struct TcPass {
   int kind;          // 0 = radial gate (A = hidden layer), 1 = SO(2) block
   int block;         // |m| of the SO(2) block
-  int n;             // accumulator columns (<= 512, multiple of 32)
+  int n;             // accumulator columns (<= 256, multiple of 32)
   int n_off;         // first output row of the block matrix covered by this pass
   int nk;            // K chunks of 64
   int last_of_kind;  // last gate pass / last pass of block 0
@@ -64,7 +64,7 @@ struct TcParams {
   int nch;
   int xbase[3];
   int npass;
-  TcPass pass[16];
+  TcPass pass[32];
   int woff[8];
   int ybase[3];
 };
@@ -75,6 +75,19 @@ struct TcWeights {
 };
 
 constexpr int kTcMaxGrid = 160;
+
+// SO(2) GEMM pass width in TMEM columns: 512 = one accumulator per pass (fewer A
+// re-reads, drain between passes), 256 = two alternating accumulators (drain overlaps
+// the next pass).  Attention logits: in the GEMM epilogue (1) or a separate kernel (0).
+#ifndef EGNN_ACC_COLS
+#define EGNN_ACC_COLS 256
+#endif
+#ifndef EGNN_LOGITS_IN_EPILOGUE
+#define EGNN_LOGITS_IN_EPILOGUE 0
+#endif
+constexpr int kTcAccCols = EGNN_ACC_COLS;
+constexpr int kTcPairRows = kTcAccCols / 2;   // label / output rows per half of a |m| > 0 pass
+constexpr bool kTcLogitsInEpilogue = EGNN_LOGITS_IN_EPILOGUE != 0;
 constexpr int kTcChunkTiles = 4096;   // edge tiles per launch range (bounds the gate and A buffers)
 
 // Tiles per launch range: the fewest ranges of at most kTcChunkTiles, balanced.

@@ -247,7 +247,13 @@ def main():
             egnn.hamiltonian_blocks(g, desc, head_w, w.shells, x, blocks, workspace=ws_head)
         return x
 
-    launches_per_step = 7 + w.n_layers + (1 if has_head else 0)
+    # Our kernels per step (tensor-core path): graph build 7 (cell_assign, scan, cell_fill,
+    # nbr_count, scan, nbr_fill, wigner); per layer a_to_f32, to_f16, prep_weights, then
+    # gate + rotate + so2_gemm per range of edge tiles, logits, agg; the head to_f16,
+    # prep_weights, the three per range, head_label.
+    n_tiles = (E + 127) // 128
+    n_ranges = max(1, -(-n_tiles // 4096))
+    launches_per_step = 7 + w.n_layers * (5 + 3 * n_ranges) + ((3 + 3 * n_ranges) if has_head else 0)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -293,7 +299,7 @@ def main():
     achieved = flops / layer_avg_s / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     traffic, traffic_note = measured_layer_traffic(E)
-    roofline = {"bound": "tensor", "kernel": "egnn_layer_forward (prep, to_f16, so2_tc, logits, agg)",
+    roofline = {"bound": "tensor", "kernel": "egnn_layer_forward (prep, to_f16, gate, rotate, so2_gemm, logits, agg)",
                 "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "traffic_note": traffic_note,
                 "peak_source": f"bf16_tflops_sustained ({peak_src})",

@@ -35,7 +35,7 @@ struct TcParams {
   const float* wig;
   const __nv_bfloat16* node_in;
   __nv_bfloat16* node_out;
-  __half* node_h;                // fp16 copy of node_in (exact), read by the A producers
+  __half* node_h;                // fp16 copy of node_in (exact), read by the rotate kernel
   const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
   const uint8_t* wprep;
   long long wprep_bytes;

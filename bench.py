@@ -36,6 +36,25 @@ import synth  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def so2_flops_per_edge(w) -> float:
+    """Algorithmic work of the SO(2) linear alone per edge (m = 0 block and the (+m, -m)
+    pairs, each pair four products of (n_m C) x (n_m 2C)), x2 FLOP."""
+    L, C = w.lmax + 1, w.channels
+    macs = (L * C) * (L * 2 * C)
+    for m in range(1, w.mmax + 1):
+        nm = L - m
+        macs += 4 * (nm * C) * (nm * 2 * C)
+    return 2.0 * macs
+
+
+def reduce_ranks(dist, dev, x: float, op: str) -> float:
+    """Max or sum of a per-rank scalar over all ranks (float64)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def layer_flops_per_edge(w) -> float:
     """Algorithmic multiply-add work of one layer per edge (radial MLP + SO(2) linear), x2 FLOP."""
     L, C, K = w.lmax + 1, w.channels, w.n_rbf
@@ -47,6 +66,23 @@ def layer_flops_per_edge(w) -> float:
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_traffic_hfo2_3000.json")
+
+
+def measured_gemm_traffic(edges_per_launch: float):
+    """DRAM bytes of one SO(2) GEMM launch from the committed ncu capture, scaled by the
+    launch's edges, or None if the kernel sources changed since the counters were taken."""
+    import hashlib
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    d = json.load(open(TRAFFIC_FILE))
+    h = hashlib.sha1()
+    for f in d["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != d["sources_sha1"]:
+        return None, "kernel sources changed since the capture"
+    gb = sum(k["read_gb"] + k["write_gb"] for k in d["kernels"] if k["kernel"].startswith("so2_gemm"))
+    per_edge = gb * 1e9 / d["edges"]
+    return per_edge * edges_per_launch, f"so2_gemm bytes per edge from {d['workload']} ({d['edges']} edges) x edges per launch"
 
 
 def measured_layer_traffic(n_edges: int):
@@ -271,40 +307,55 @@ def main():
     time.sleep(0.3)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    egnn.profile(True)   # CUDA events around each SO(2) GEMM launch, on its own stream
     t_start.record(stream)
     for _ in range(args.steps):
         step(record_layers=True)
     t_end.record(stream)
     torch.cuda.synchronize()
+    egnn.profile(False)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     layer_ms = [a.elapsed_time(b) for a, b in ev_layer]
+    gemm_ms, gemm_n, gemm_edges = egnn.profile_read()
     if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        tot_e = torch.tensor([float(E)], device=dev)
-        dist.all_reduce(tot_e, op=dist.ReduceOp.SUM)
-        edges_all = float(tot_e.item())
+        total_ms = reduce_ranks(dist, dev, total_ms, "max")
+        edges_all = reduce_ranks(dist, dev, float(E), "sum")
     else:
         edges_all = float(E)
     value = edges_all * w.n_layers * args.steps / (total_ms / 1e3)
 
-    # ---- roofline of the dominant kernel (the layer) ----
+    # ---- roofline of the dominant kernel: the SO(2) GEMM (tcgen05) ----
     peaks, peak_src = load_peaks()
-    layer_avg_s = (sum(layer_ms) / len(layer_ms)) / 1e3
-    flops = layer_flops_per_edge(w) * E
-    achieved = flops / layer_avg_s / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    traffic, traffic_note = measured_layer_traffic(E)
-    roofline = {"bound": "tensor", "kernel": "egnn_layer_forward (prep, to_f16, gate, rotate, so2_gemm, logits, agg)",
-                "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic, "traffic_note": traffic_note,
-                "peak_source": f"bf16_tflops_sustained ({peak_src})",
-                "flops_per_launch": flops, "layer_ms": 1e3 * layer_avg_s,
-                "layer_edges_per_s": E / layer_avg_s}
+    layer_avg_s = (sum(layer_ms) / len(layer_ms)) / 1e3
+    layer_flops = layer_flops_per_edge(w) * E
+    layer_tf = layer_flops / layer_avg_s / 1e12
+    if gemm_n > 0:
+        per_launch_edges = gemm_edges / gemm_n
+        gemm_flops = so2_flops_per_edge(w) * per_launch_edges
+        gemm_avg_s = gemm_ms / gemm_n / 1e3
+        achieved = gemm_flops / gemm_avg_s / 1e12
+        traffic, traffic_note = measured_gemm_traffic(per_launch_edges)
+        roofline = {"bound": "tensor", "kernel": "so2_gemm_kernel (SO(2) linear on tcgen05)",
+                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": traffic, "traffic_note": traffic_note,
+                    "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                    "flops_per_launch": gemm_flops, "launch_ms": 1e3 * gemm_avg_s, "launches": gemm_n,
+                    "edges_per_launch": per_launch_edges,
+                    "timing": "CUDA events recorded by the library around each launch, on its stream, "
+                              "inside the timed region"}
+    else:
+        traffic, traffic_note = measured_layer_traffic(E)
+        roofline = {"bound": "tensor", "kernel": "egnn_layer_forward", "achieved": layer_tf, "peak": peak,
+                    "unit": "TFLOP/s", "frac": layer_tf / peak, "traffic": traffic, "traffic_note": traffic_note,
+                    "peak_source": f"bf16_tflops_sustained ({peak_src})", "flops_per_launch": layer_flops}
+    roofline["layer_call"] = {"kernels": "a_to_f32, to_f16, prep_weights, (gate, rotate, so2_gemm) per edge-tile "
+                                         "range, logits, agg",
+                              "ms": 1e3 * layer_avg_s, "tflops": layer_tf, "frac": layer_tf / peak,
+                              "flops_per_call": layer_flops, "edges_per_s": E / layer_avg_s}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -330,9 +381,7 @@ def main():
             torch.cuda.synchronize()
         t_e2e = time.perf_counter() - t0
         if world > 1:
-            t = torch.tensor([t_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e2e = float(t.item())
+            t_e2e = reduce_ranks(dist, dev, t_e2e, "max")
         e2e = {"value": edges_all * w.n_layers * e2e_steps / t_e2e, "unit": "edges/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "note": "pinned host inputs (positions, species, embeddings) -> full step -> blocks to host; "

@@ -514,6 +514,20 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
   return EGNN_OK;
 }
 
+extern "C" egnn_status egnn_profile(int32_t enable) {
+  tc_profile_enable(enable != 0);
+  return EGNN_OK;
+}
+
+extern "C" egnn_status egnn_profile_read(double* gemm_ms, int64_t* launches, int64_t* edges) {
+  if (!gemm_ms || !launches || !edges) return EGNN_ERR_INVALID_ARG;
+  long long n = 0, e = 0;
+  EGNN_CUDA_TRY(tc_profile_read(gemm_ms, &n, &e));
+  *launches = n;
+  *edges = e;
+  return EGNN_OK;
+}
+
 extern "C" egnn_status egnn_read_status(const egnn_graph* g, int32_t* code, void* cuda_stream) {
   if (!g || !g->status) return EGNN_ERR_INVALID_ARG;
   int32_t v = 0;

@@ -1184,6 +1184,40 @@ __global__ void a_to_f32_kernel(const __nv_bfloat16* __restrict__ A, float* __re
   if (i < n) out[i] = __bfloat162float(A[i]);
 }
 
+// ---- opt-in timing of the SO(2) GEMM launches of layer calls (diagnostics) ----
+// While enabled, each so2_gemm launch of a layer call is bracketed by two CUDA events
+// recorded on its own stream; the events are created once, on first use, and kept.
+constexpr int kProfMax = 4096;
+static bool g_prof_on = false;
+static int g_prof_n = 0;
+static long long g_prof_edges = 0;
+static cudaEvent_t g_prof_ev[2][kProfMax];
+static bool g_prof_made[kProfMax];
+
+void tc_profile_enable(bool on) {
+  g_prof_on = on;
+  if (on) {
+    g_prof_n = 0;
+    g_prof_edges = 0;
+  }
+}
+
+cudaError_t tc_profile_read(double* ms, long long* launches, long long* edges) {
+  double tot = 0.0;
+  for (int i = 0; i < g_prof_n; ++i) {
+    cudaError_t e = cudaEventSynchronize(g_prof_ev[1][i]);
+    if (e != cudaSuccess) return e;
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, g_prof_ev[0][i], g_prof_ev[1][i]);
+    if (e != cudaSuccess) return e;
+    tot += t;
+  }
+  *ms = tot;
+  *launches = g_prof_n;
+  *edges = g_prof_edges;
+  return cudaSuccess;
+}
+
 template <int LM, int MM>
 static void launch_rotate(const TcParams& P, int nt, cudaStream_t st) {
   rotate_kernel<LM, MM><<<nt, 256, 0, st>>>(P);
@@ -1245,8 +1279,24 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
     gate_kernel<<<grid, kThreads, sm_g, st>>>(Pg);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if ((err = launch_rotate_any(Ps, nt, st)) != cudaSuccess) return err;
+    const int pi = g_prof_n;
+    const bool prof = g_prof_on && P.with_logits && !P.label_mode && pi < kProfMax;
+    if (prof) {
+      if (!g_prof_made[pi]) {
+        if ((err = cudaEventCreate(&g_prof_ev[0][pi])) != cudaSuccess) return err;
+        if ((err = cudaEventCreate(&g_prof_ev[1][pi])) != cudaSuccess) return err;
+        g_prof_made[pi] = true;
+      }
+      if ((err = cudaEventRecord(g_prof_ev[0][pi], st)) != cudaSuccess) return err;
+    }
     so2_gemm_kernel<<<grid, kGThreads, sm_s, st>>>(Ps);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (prof) {
+      if ((err = cudaEventRecord(g_prof_ev[1][pi], st)) != cudaSuccess) return err;
+      const long long e_end = (long long)te * 128 < P.n_edges ? (long long)te * 128 : P.n_edges;
+      g_prof_edges += e_end - (long long)tb * 128;
+      g_prof_n = pi + 1;
+    }
   }
   return cudaSuccess;
 }

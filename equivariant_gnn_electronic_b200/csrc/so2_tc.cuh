@@ -107,3 +107,5 @@ cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t 
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
                            float* blocks, cudaStream_t st);
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te);
+void tc_profile_enable(bool on);
+cudaError_t tc_profile_read(double* ms, long long* launches, long long* edges);

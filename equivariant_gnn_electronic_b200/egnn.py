@@ -23,6 +23,7 @@ EGNN_WS_BUILD_GRAPH, EGNN_WS_LAYER, EGNN_WS_HAMILTONIAN = 0, 1, 2
 EXPORTED = (
     "egnn_wigner_floats", "egnn_workspace_bytes", "egnn_build_graph", "egnn_layer_forward",
     "egnn_hamiltonian_blocks", "egnn_read_status", "egnn_status_string", "egnn_build_graph_noalloc",
+    "egnn_profile", "egnn_profile_read",
 )
 
 
@@ -70,6 +71,10 @@ def _load():
     lib.egnn_read_status.restype = i32
     lib.egnn_status_string.argtypes = [i32]
     lib.egnn_status_string.restype = ctypes.c_char_p
+    lib.egnn_profile.argtypes = [i32]
+    lib.egnn_profile.restype = i32
+    lib.egnn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    lib.egnn_profile_read.restype = i32
     return lib
 
 
@@ -93,6 +98,18 @@ def _stream(stream) -> int:
 
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def profile(enable: bool) -> None:
+    """Start (clearing the record) or stop timing the SO(2) GEMM launches of layer calls."""
+    _check(lib.egnn_profile(1 if enable else 0), "egnn_profile")
+
+
+def profile_read() -> tuple[float, int, int]:
+    """(summed GEMM launch milliseconds, launches, edges processed) of the record."""
+    ms, n, e = ctypes.c_double(0.0), ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib.egnn_profile_read(ctypes.byref(ms), ctypes.byref(n), ctypes.byref(e)), "egnn_profile_read")
+    return ms.value, n.value, e.value
 
 
 def wigner_floats(lmax: int, mmax: int) -> int:

@@ -193,6 +193,22 @@ egnn_status egnn_read_status(const egnn_graph* g, int32_t* code, void* cuda_stre
 /* Short text for a status value (static storage). */
 const char* egnn_status_string(egnn_status s);
 
+/*
+ * egnn_profile / egnn_profile_read -- opt-in timing of the SO(2) GEMM kernel of
+ * tensor-core egnn_layer_forward calls (a diagnostic; the pages have no counterpart).
+ * egnn_profile(1) clears the record and starts recording; egnn_profile(0) stops.
+ * While recording, every SO(2) GEMM launch of a layer call is bracketed by two CUDA
+ * events recorded on that call's stream (at most 4096 launches per record; later
+ * ones are not recorded).  The events are created on first use, on the device
+ * current at the time, and kept until the process exits: use one device per
+ * process.  Not thread-safe.  Head calls and the SIMT path are not recorded.
+ * egnn_profile_read waits for the recorded events and returns the summed launch
+ * time in milliseconds, the number of launches and the number of edges they
+ * processed; null outputs return EGNN_ERR_INVALID_ARG, a CUDA error EGNN_ERR_CUDA.
+ */
+egnn_status egnn_profile(int32_t enable);
+egnn_status egnn_profile_read(double* gemm_ms, int64_t* launches, int64_t* edges);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,3 +77,10 @@ def test_argument_checks_return_before_any_launch():
     ws = 1 << 20
     assert lib.egnn_hamiltonian_blocks(ctypes.byref(g), ctypes.byref(d), fake, sh, 2, fake, fake, fake, ws,
                                        None) == egnn.EGNN_ERR_UNSUPPORTED
+
+
+def test_profile_record_starts_empty_and_checks_outputs():
+    egnn.profile(True)
+    egnn.profile(False)
+    assert egnn.profile_read() == (0.0, 0, 0)
+    assert egnn.lib.egnn_profile_read(None, None, None) == egnn.EGNN_ERR_INVALID_ARG

@@ -789,32 +789,55 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
 
 
 // Attention logits a_{e,h} = A[h] . SiLU(y0_e) + bA[h], one warp per edge: lanes
-// read y0 (fp32, coalesced) and the fp32 copy of A staged in shared memory, then the
-// heads' partial sums are reduced across the warp.
+// read y0 (fp32, coalesced) and A from shared memory, stored column-major with a
+// column's heads contiguous (stride HS = 4 ceil(H/4) + 4 floats: 16-byte aligned and
+// free of bank conflicts for eight lanes' 16-byte reads), so one 16-byte read serves
+// four heads; the next edge's y0 is loaded while this edge is reduced; the heads'
+// partial sums are then reduced across the warp.
 __global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcParams P) {
-  extern __shared__ float As[];                 // [H][L*C]
-  const int LC = P.L * P.C, H = P.H;
-  for (int i = threadIdx.x; i < H * LC; i += blockDim.x) As[i] = P.Af[i];
+  extern __shared__ float As[];                 // [L*C][HS]
+  const int LC = P.L * P.C, H = P.H, HQ = (H + 3) >> 2, HS = 4 * HQ + 4;
+  for (int i = threadIdx.x; i < LC * HS; i += blockDim.x) {
+    const int j = i / HS, h = i - j * HS;
+    As[i] = h < H ? P.Af[h * LC + j] : 0.f;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < P.n_edges; e += nw) {
+  long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  float yv[28];                                  // LC <= 7 * 128 = 896 = 28 * 32
+  if (e < P.n_edges) {
     const float* y0 = reinterpret_cast<const float*>(P.Y + e * (long long)P.y_row_bytes);
+#pragma unroll
+    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
+  }
+  for (; e < P.n_edges; e += nw) {
     float a[16];
 #pragma unroll
     for (int h = 0; h < 16; ++h) a[h] = 0.f;
-    float yv[28];                                // LC <= 7 * 128 = 896 = 28 * 32: all loads first
-#pragma unroll
-    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
 #pragma unroll
     for (int k = 0; k < 28; ++k) {
       const int j = lane + 32 * k;
       if (j < LC) {
         const float sv = yv[k] / (1.0f + __expf(-yv[k]));
+        const float4* ap = reinterpret_cast<const float4*>(As + j * HS);
 #pragma unroll
-        for (int h = 0; h < 16; ++h)
-          if (h < H) a[h] += As[h * LC + j] * sv;
+        for (int q = 0; q < 4; ++q) {
+          if (q < HQ) {
+            const float4 w = ap[q];
+            a[4 * q] += w.x * sv;
+            a[4 * q + 1] += w.y * sv;
+            a[4 * q + 2] += w.z * sv;
+            a[4 * q + 3] += w.w * sv;
+          }
+        }
       }
+    }
+    const long long en = e + nw;
+    if (en < P.n_edges) {
+      const float* y0 = reinterpret_cast<const float*>(P.Y + en * (long long)P.y_row_bytes);
+#pragma unroll
+      for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
     }
 #pragma unroll
     for (int h = 0; h < 16; ++h) {
@@ -1353,7 +1376,7 @@ cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t 
   cudaError_t err = launch_tc_gemm(P, W, st);
   if (err != cudaSuccess) return err;
   if (!kTcLogitsInEpilogue && P.n_edges > 0) {
-    const size_t sm = sizeof(float) * (size_t)P.H * P.L * P.C;
+    const size_t sm = sizeof(float) * (size_t)(4 * ((P.H + 3) / 4) + 4) * P.L * P.C;
     err = cudaFuncSetAttribute(logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (err != cudaSuccess) return err;
     int nb = 2;

@@ -26,10 +26,11 @@
 //                 alternating TMEM accumulators, with B = W0 (|m| = 0) or
 //                 [W_b1 ; W_b2] read by four MMAs, one with the negate-B bit, per K
 //                 block (|m| = b > 0); the epilogue writes y_e (y0 in fp32, |m| > 0
-//                 in bf16) and the attention logits A SiLU(y0_e) + bA, or, for the
-//                 head, edge-frame labels.
-//   Then agg (one CTA per destination atom: softmax over its incoming edges, rotate
-//   back with the kept rows of D^l, weighted sum, residual; no atomics).
+//                 in bf16) or, for the head, edge-frame labels (with
+//                 kTcLogitsInEpilogue it also forms the attention logits).
+//   Then logits (a_e = A SiLU(y0_e) + bA, warp per edge) and agg (one CTA per
+//   destination atom: softmax over its incoming edges, rotate back with the kept
+//   rows of D^l, weighted sum, residual; no atomics).
 #include <math.h>
 
 #include "common.cuh"

@@ -36,17 +36,23 @@ def _nvcc() -> str:
 def build(verbose: bool = False, force: bool = False) -> str:
     os.makedirs(BUILD_DIR, exist_ok=True)
     nvcc = _nvcc()
+    from concurrent.futures import ThreadPoolExecutor
+
     objs = []
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(ROOT, "include", "egnn.h")]
     newest_dep = max(os.path.getmtime(p) for p in deps)
+    todo = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
         o = os.path.join(BUILD_DIR, src + ".o")
         objs.append(o)
         if not force and os.path.exists(o) and os.path.getmtime(o) >= newest_dep:
             continue
-        cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-c", s, "-o", o]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        todo.append((src, [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-c", s, "-o", o]))
+    # one nvcc per translation unit, run side by side
+    with ThreadPoolExecutor(max_workers=max(1, len(todo))) as ex:
+        results = list(ex.map(lambda t: (t[0], subprocess.run(t[1], capture_output=True, text=True)), todo))
+    for src, r in results:
         if verbose or r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:

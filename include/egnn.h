@@ -84,7 +84,11 @@ int32_t egnn_wigner_floats(int32_t lmax, int32_t mmax);
 enum { EGNN_WS_BUILD_GRAPH = 0, EGNN_WS_LAYER = 1, EGNN_WS_HAMILTONIAN = 2 };
 
 /* Bytes of device workspace `which` needs (0 allowed).  For EGNN_WS_BUILD_GRAPH
- * only n_atoms matters and desc may be NULL. */
+ * only n_atoms matters and desc may be NULL.  For the tensor-core layer and head
+ * (bf16, C = 128) the size grows with n_edges by the per-edge message record
+ * (4 L C + 4 C sum_{b=1..mmax} (L - b) bytes, 6 KB at lmax 4, mmax 2) plus 4 bytes per
+ * edge and head for the attention logits; the gate and A-operand buffers are sized
+ * for one range of at most 4096 edge tiles of 128 edges and stop growing beyond it. */
 size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* desc, int32_t n_atoms,
                             int64_t n_edges);
 

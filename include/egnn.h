@@ -176,7 +176,10 @@ egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_desc* desc,
  * with one k per shell pair (a, b) containing L (pairs lexicographic, a outer);
  * block[(a,i),(b,j)] = sum_{L,M} C^L_{(l_a i)(l_b j),M} h[L,M,k(a,b,L)], where C^L
  * is the real Clebsch-Gordan matrix of the basis above (orthonormal columns,
- * first non-zero entry of column M=-L positive).
+ * first non-zero entry of column M=-L positive).  The tensor-core path applies U^L
+ * in the edge frame (U^L folded into the SO(2) weights, then the labels rotated
+ * back), which equals the order above up to rounding because U^L mixes channels
+ * only and the rotation mixes m only.
  * head_weights device, packed like a layer's W1..Wm2 (no A, bA), then U^L[mult_L][C]
  *   for L = 0..lmax (absent when mult_L = 0).
  * shell_l   host int32 [n_shells]: orbital template shared by all species,

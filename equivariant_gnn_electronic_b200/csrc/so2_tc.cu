@@ -91,15 +91,31 @@ __device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& 
   if (ps.kind == 1 && ps.block > 0 && !P.label_mode && g >= ps.np)
     col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
   float4* srow = reinterpret_cast<float4*>(st + lane * 36);
+  // gate passes: the group's 32 b2 values (bf16, 64 bytes, 16-byte aligned), all
+  // loaded through the read-only path before any store
+  uint32_t bw[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) bw[k] = 0u;
+  if (ps.kind == 0) {
+    const uint4* bp = reinterpret_cast<const uint4*>(P.b2 + col);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = __ldg(bp + k);
+      bw[4 * k] = w.x;
+      bw[4 * k + 1] = w.y;
+      bw[4 * k + 2] = w.z;
+      bw[4 * k + 3] = w.w;
+    }
+  }
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     float4 x = make_float4(__uint_as_float(ru[4 * q]), __uint_as_float(ru[4 * q + 1]),
                            __uint_as_float(ru[4 * q + 2]), __uint_as_float(ru[4 * q + 3]));
-    if (ps.kind == 0) {
-      x.x += __bfloat162float(P.b2[col + 4 * q]);
-      x.y += __bfloat162float(P.b2[col + 4 * q + 1]);
-      x.z += __bfloat162float(P.b2[col + 4 * q + 2]);
-      x.w += __bfloat162float(P.b2[col + 4 * q + 3]);
+    if (ps.kind == 0) {   // bf16 pair (lo, hi) -> fp32 by placing each in the high half
+      x.x += __uint_as_float(bw[2 * q] << 16);
+      x.y += __uint_as_float(bw[2 * q] & 0xffff0000u);
+      x.z += __uint_as_float(bw[2 * q + 1] << 16);
+      x.w += __uint_as_float(bw[2 * q + 1] & 0xffff0000u);
     }
     srow[q] = x;
   }

@@ -122,6 +122,23 @@ def test_layer_bf16_degrees(egnn, lmax, mmax):
     check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"])
 
 
+@pytest.mark.parametrize("heads", [1, 16])
+def test_layer_bf16_head_counts(egnn, heads):
+    # tensor-core layer at the fewest and the most attention heads it accepts
+    w = dataclasses.replace(synth.WORKLOADS["hfo2_3000"], heads=heads)
+    pos, _, box = cell("hfo2_3000", 0, 100)
+    g = gpu_graph(egnn, "hfo2_3000", 0, 100)
+    desc = egnn.desc_for(w)
+    n = synth.make_embeddings(w, len(pos), 0)
+    W = synth.make_layer_weights(w, 0, bias_std=0.1)
+    out = egnn.layer_forward(g, desc, egnn.pack_weights(W, desc), to_dev(n, torch.bfloat16))
+    torch.cuda.synchronize()
+    assert g.read_status() == 0
+    rp, src, sh = oracle_graph("hfo2_3000", 0, 100)
+    ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
+    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"])
+
+
 def test_layer_is_deterministic(egnn):
     w = synth.WORKLOADS["hfo2_3000"]
     pos, species, box = cell("hfo2_3000", 0, 300)

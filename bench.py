@@ -65,40 +65,71 @@ def layer_flops_per_edge(w) -> float:
     return 2.0 * macs
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_traffic_hfo2_3000.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_traffic_gst_8064.json")
+TRAFFIC_SOURCES = ["equivariant_gnn_electronic_b200/csrc/so2_fused.cu", "equivariant_gnn_electronic_b200/csrc/so2_tc.cu",
+                   "equivariant_gnn_electronic_b200/csrc/so2_tc.cuh", "equivariant_gnn_electronic_b200/csrc/tc_ptx.cuh",
+                   "equivariant_gnn_electronic_b200/csrc/api.cu"]
+LAYER_KERNELS = ("prep_weights", "gate_kernel", "rotate_kernel", "layer_fused_kernel", "combine_kernel")
 
 
-def measured_gemm_traffic(edges_per_launch: float):
-    """DRAM bytes of one SO(2) GEMM launch from the committed ncu capture, scaled by the
-    launch's edges, or None if the kernel sources changed since the counters were taken."""
+def sources_sha1() -> str:
     import hashlib
+    h = hashlib.sha1()
+    for f in TRAFFIC_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
+
+
+def ingest_traffic(csv_path: str, workload: str, edges: int) -> None:
+    """Writes the per-kernel DRAM traffic record of one layer call from an ncu CSV (metrics
+    dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum; one capture of the
+    layer call's launches), stamped with the hash of the kernel sources it was taken on."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hdr = next(i for i, r in enumerate(rows) if "Kernel Name" in r and "Metric Name" in r)
+    cols = rows[hdr]
+    ki, mi, vi, ui = cols.index("Kernel Name"), cols.index("Metric Name"), cols.index("Metric Value"), \
+        cols.index("Metric Unit")
+    idi = cols.index("ID")
+    launches = {}
+    for r in rows[hdr + 1:]:
+        if len(r) <= max(ki, mi, vi, ui):
+            continue
+        name = next((k for k in LAYER_KERNELS if k in r[ki]), None)
+        if name is None:
+            continue
+        v = float(r[vi].replace(",", ""))
+        unit = r[ui].lower()
+        scale = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "nsecond": 1e-6, "usecond": 1e-3,
+                 "msecond": 1.0}.get(unit, 1.0)
+        launches.setdefault((r[idi], name), {})[r[mi]] = v * scale
+    per = {}
+    for (_, name), m in launches.items():
+        k = per.setdefault(name, {"kernel": name, "launches": 0, "read_gb": 0.0, "write_gb": 0.0, "ms": 0.0})
+        k["launches"] += 1
+        k["read_gb"] += m.get("dram__bytes_read.sum", 0.0) / 1e9
+        k["write_gb"] += m.get("dram__bytes_write.sum", 0.0) / 1e9
+        k["ms"] += m.get("gpu__time_duration.sum", 0.0)
+    tot = sum(k["read_gb"] + k["write_gb"] for k in per.values())
+    rec = {"workload": workload, "edges": edges, "sources": TRAFFIC_SOURCES, "sources_sha1": sources_sha1(),
+           "kernels": list(per.values()), "bytes_per_edge": tot * 1e9 / edges,
+           "note": "one ncu capture of one layer call; counters from a single pass per launch"}
+    json.dump(rec, open(TRAFFIC_FILE, "w"), indent=1)
+    print(json.dumps(rec, indent=1))
+
+
+def measured_traffic(kernel_prefix=None):
+    """DRAM bytes per edge of the dominant kernel (or, without a prefix, of the whole layer
+    call) from the committed capture, or None if the kernel sources changed since."""
     if not os.path.exists(TRAFFIC_FILE):
         return None, "no capture"
     d = json.load(open(TRAFFIC_FILE))
-    h = hashlib.sha1()
-    for f in d["sources"]:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
-    if h.hexdigest() != d["sources_sha1"]:
+    if d.get("sources_sha1") != sources_sha1():
         return None, "kernel sources changed since the capture"
-    gb = sum(k["read_gb"] + k["write_gb"] for k in d["kernels"] if k["kernel"].startswith("so2_gemm"))
-    per_edge = gb * 1e9 / d["edges"]
-    return per_edge * edges_per_launch, f"so2_gemm bytes per edge from {d['workload']} ({d['edges']} edges) x edges per launch"
-
-
-def measured_layer_traffic(n_edges: int):
-    """DRAM bytes of one layer call from the committed ncu capture, scaled to n_edges by the
-    edge count (the traffic grows with the edges), or None if the kernel sources changed
-    since the counters were taken."""
-    import hashlib
-    if not os.path.exists(TRAFFIC_FILE):
-        return None, "no capture"
-    d = json.load(open(TRAFFIC_FILE))
-    h = hashlib.sha1()
-    for f in d["sources"]:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
-    if h.hexdigest() != d["sources_sha1"]:
-        return None, "kernel sources changed since the capture"
-    return d["bytes_per_edge"] * n_edges, f"scaled from {d['workload']} ({d['edges']} edges) by edge count"
+    if kernel_prefix is None:
+        return d["bytes_per_edge"], f"layer call, from {d['workload']} ({d['edges']} edges)"
+    gb = sum(k["read_gb"] + k["write_gb"] for k in d["kernels"] if k["kernel"].startswith(kernel_prefix))
+    return gb * 1e9 / d["edges"], f"{kernel_prefix} bytes per edge from {d['workload']} ({d['edges']} edges)"
 
 
 def load_peaks():
@@ -178,6 +209,15 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_baseline(w, pos, box, n_emb, W, atoms):
+    """The oracle on this host: the same sample on every BLAS thread, then on one thread."""
+    from threadpoolctl import threadpool_limits
+    ne, t_all, graph = oracle_sample_run(w, pos, box, n_emb, W, atoms)
+    with threadpool_limits(limits=1):
+        _, t_one, _ = oracle_sample_run(w, pos, box, n_emb, W, atoms, graph)
+    return ne, t_all, t_one
+
+
 def run_reference(args, w):
     """The oracle on this host's cores: each step = the layer over a bounded atom sample."""
     pos, species, box = synth.make_cell(w, 0)
@@ -220,8 +260,14 @@ def main():
     ap.add_argument("--ref-atoms", type=int, default=256)
     ap.add_argument("--cpu-atoms", type=int, default=160, help="oracle sample for cpu_baseline (0: skip)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ingest-traffic", default=None,
+                    help="ncu CSV of one layer call: write the DRAM traffic record for the workload and exit")
+    ap.add_argument("--edges", type=int, default=0, help="edges of the captured layer call (with --ingest-traffic)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.ingest_traffic:
+        ingest_traffic(args.ingest_traffic, w.name, args.edges)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -284,12 +330,12 @@ def main():
         return x
 
     # Our kernels per step (tensor-core path): graph build 7 (cell_assign, scan, cell_fill,
-    # nbr_count, scan, nbr_fill, wigner); per layer a_to_f32, to_f16, prep_weights, then
-    # gate + rotate + so2_gemm per range of edge tiles, logits, agg; the head to_f16,
-    # prep_weights, the three per range, head_label.
+    # nbr_count, scan, nbr_fill, wigner); per layer prep_weights, then gate + rotate +
+    # layer_fused per range of edge tiles, then combine; the head prep_weights, gate +
+    # rotate + so2_gemm per range, head_label.
     n_tiles = (E + 127) // 128
     n_ranges = max(1, -(-n_tiles // 4096))
-    launches_per_step = 7 + w.n_layers * (5 + 3 * n_ranges) + ((3 + 3 * n_ranges) if has_head else 0)
+    launches_per_step = 7 + w.n_layers * (2 + 3 * n_ranges) + ((2 + 3 * n_ranges) if has_head else 0)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -327,35 +373,39 @@ def main():
         edges_all = float(E)
     value = edges_all * w.n_layers * args.steps / (total_ms / 1e3)
 
-    # ---- roofline of the dominant kernel: the SO(2) GEMM (tcgen05) ----
+    # ---- roofline of the dominant kernel: the fused layer kernel (tcgen05) ----
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     layer_avg_s = (sum(layer_ms) / len(layer_ms)) / 1e3
     layer_flops = layer_flops_per_edge(w) * E
     layer_tf = layer_flops / layer_avg_s / 1e12
-    if gemm_n > 0:
-        per_launch_edges = gemm_edges / gemm_n
-        gemm_flops = so2_flops_per_edge(w) * per_launch_edges
-        gemm_avg_s = gemm_ms / gemm_n / 1e3
-        achieved = gemm_flops / gemm_avg_s / 1e12
-        traffic, traffic_note = measured_gemm_traffic(per_launch_edges)
-        roofline = {"bound": "tensor", "kernel": "so2_gemm_kernel (SO(2) linear on tcgen05)",
-                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": traffic, "traffic_note": traffic_note,
-                    "peak_source": f"bf16_tflops_sustained ({peak_src})",
-                    "flops_per_launch": gemm_flops, "launch_ms": 1e3 * gemm_avg_s, "launches": gemm_n,
-                    "edges_per_launch": per_launch_edges,
-                    "timing": "CUDA events recorded by the library around each launch, on its stream, "
-                              "inside the timed region"}
-    else:
-        traffic, traffic_note = measured_layer_traffic(E)
-        roofline = {"bound": "tensor", "kernel": "egnn_layer_forward", "achieved": layer_tf, "peak": peak,
-                    "unit": "TFLOP/s", "frac": layer_tf / peak, "traffic": traffic, "traffic_note": traffic_note,
-                    "peak_source": f"bf16_tflops_sustained ({peak_src})", "flops_per_launch": layer_flops}
-    roofline["layer_call"] = {"kernels": "a_to_f32, to_f16, prep_weights, (gate, rotate, so2_gemm) per edge-tile "
-                                         "range, logits, agg",
+    per_edge_traffic, traffic_note = measured_traffic("layer_fused")
+    layer_traffic, layer_traffic_note = measured_traffic(None)
+    per_launch_edges = gemm_edges / gemm_n if gemm_n else float(E)
+    gemm_flops = so2_flops_per_edge(w) * per_launch_edges
+    gemm_avg_s = gemm_ms / gemm_n / 1e3 if gemm_n else layer_avg_s
+    achieved = gemm_flops / gemm_avg_s / 1e12
+    roofline = {"bound": "tensor",
+                "kernel": "layer_fused_kernel (SO(2) linear on tcgen05 with the attention logits, "
+                          "per-atom softmax, rotate-back and aggregation in its epilogue)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "frac_of_burst": achieved / peak_burst,
+                "traffic": None if per_edge_traffic is None else per_edge_traffic * per_launch_edges,
+                "traffic_note": traffic_note,
+                "peak_source": f"bf16_tflops_sustained ({peak_src}); burst {peak_burst}",
+                "flops_per_launch": gemm_flops, "flops_counted": "SO(2) blocks only, 8.19 MFLOP per edge at lmax 4",
+                "launch_ms": 1e3 * gemm_avg_s, "launches": gemm_n, "edges_per_launch": per_launch_edges,
+                "timing": "CUDA events recorded by the library around each launch, on its stream, "
+                          "inside the timed region",
+                "messages_in_hbm": False}
+    roofline["layer_call"] = {"kernels": "prep_weights, (gate, rotate, layer_fused) per edge-tile range, combine",
                               "ms": 1e3 * layer_avg_s, "tflops": layer_tf, "frac": layer_tf / peak,
-                              "flops_per_call": layer_flops, "edges_per_s": E / layer_avg_s}
+                              "frac_of_burst": layer_tf / peak_burst,
+                              "flops_per_call": layer_flops, "flops_counted": "radial MLP + SO(2), 8.528 MFLOP/edge",
+                              "edges_per_s": E / layer_avg_s,
+                              "traffic": None if layer_traffic is None else layer_traffic * E,
+                              "traffic_note": layer_traffic_note}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -391,9 +441,12 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and args.cpu_atoms > 0:
         atoms = np.sort(np.random.default_rng(7).choice(len(pos_np), args.cpu_atoms, replace=False))
-        ne, dts, _ = oracle_sample_run(w, pos_np, box, n_np, synth.make_layer_weights(w, 0), atoms)
-        cpu = {"value": ne / dts, "unit": "edges/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"one layer over {len(atoms)} random destination atoms ({ne} edges), fp64 numpy oracle"}
+        ne, t_all, t_one = oracle_baseline(w, pos_np, box, n_np, synth.make_layer_weights(w, 0), atoms)
+        cpu = {"value": ne / t_all, "unit": "edges/s", "cores": blas_threads(), "kind": "oracle",
+               "nproc": os.cpu_count(),
+               "single_thread": {"value": ne / t_one, "unit": "edges/s", "cores": 1},
+               "sample": f"one layer over {len(atoms)} random destination atoms ({ne} edges), fp64 numpy oracle, "
+                         f"timed on all BLAS threads and on one"}
 
     if rank == 0:
         line = {

@@ -197,7 +197,7 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
 }
 
 struct TcWorkspace {
-  size_t wprep, gate, x, y, logits, node_h, af, total;
+  size_t wprep, gate, x, y, logits, af, total;
 };
 
 TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_atoms) {
@@ -212,17 +212,47 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_at
   w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
   w.y = w.x + align_up(tch * P.nch * 16384, 1024);
   w.logits = w.y + align_up(E * (size_t)P.y_row_bytes, 1024);
-  w.node_h = w.logits + align_up(E * d->heads * 4, 1024);
-  size_t N = n_atoms > 0 ? (size_t)n_atoms : 0;
-  w.af = w.node_h + align_up(N * (d->lmax + 1) * (d->lmax + 1) * d->channels * 2, 1024);
+  (void)n_atoms;
+  w.af = w.logits + align_up(E * d->heads * 4, 1024);
   w.total = w.af + align_up((size_t)d->heads * (d->lmax + 1) * d->channels * 4, 1024) + 1024;
   return w;
 }
 
+// Workspace of the fused tensor-core layer: prepared weights, the gates and A tiles of
+// one range of edge tiles, the per-CTA y0 stash, per-atom accumulators and two
+// partial records per edge tile.  Nothing in it is stored per edge except the
+// records (2 (L^2 C + 32) floats per 128 edges).
+struct LayerWorkspace {
+  size_t wprep, gate, x, stash, acc, slots, total;
+  int rec_floats;
+};
+
+LayerWorkspace layer_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_atoms) {
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  tc_plan(d, P);
+  LayerWorkspace w;
+  const size_t E = n_edges > 0 ? (size_t)n_edges : 0, N = n_atoms > 0 ? (size_t)n_atoms : 0;
+  const size_t L = d->lmax + 1, C = d->channels;
+  const size_t n_tiles = (E + 127) / 128;
+  const size_t tch = (size_t)tc_chunk_tiles((int)n_tiles);
+  w.rec_floats = (int)(L * L * C + 32);
+  w.wprep = 0;
+  w.gate = align_up((size_t)P.wprep_bytes, 1024);
+  w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
+  w.stash = w.x + align_up(tch * P.nch * 16384, 1024);
+  w.acc = w.stash + align_up((size_t)kTcMaxGrid * L * 128 * C * 2, 1024);
+  w.slots = w.acc + align_up(N * L * L * C * 4, 1024);
+  w.total = w.slots + align_up(n_tiles * 2 * (size_t)w.rec_floats * 4, 1024) + 1024;
+  return w;
+}
+
 // Fills the tensor-core launch parameters for graph g, weights W and a 1024-aligned
-// workspace (label mode with `mult`); returns false if the pass plan does not fit.
+// workspace (label mode with `mult`; the fused layer's layout with `layer`); returns
+// false if the pass plan does not fit.
 bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_desc* desc, const So2Weights& W,
-             const void* node_in, void* node_out, uint8_t* ws, int with_logits, const int* mult = nullptr) {
+             const void* node_in, void* node_out, uint8_t* ws, int with_logits, const int* mult = nullptr,
+             bool layer = false) {
   TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
   memset(&T, 0, sizeof(T));
   if (!tc_plan(desc, T, mult)) return false;
@@ -256,13 +286,44 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   T.b2 = (const __nv_bfloat16*)W.b2;
   T.A = (const __nv_bfloat16*)W.A;
   T.bA = (const __nv_bfloat16*)W.bA;
-  T.wprep = ws + wl.wprep;
-  T.gates = (__half*)(ws + wl.gate);
-  T.X = ws + wl.x;
-  T.Y = ws + wl.y;
-  T.logits = (float*)(ws + wl.logits);
-  T.node_h = (__half*)(ws + wl.node_h);
-  T.Af = (float*)(ws + wl.af);
+  if (layer) {
+    const LayerWorkspace lw = layer_workspace(desc, g->n_edges, g->n_atoms);
+    T.wprep = ws + lw.wprep;
+    T.gates = (__nv_bfloat16*)(ws + lw.gate);
+    T.X = ws + lw.x;
+    T.stash = (__nv_bfloat16*)(ws + lw.stash);
+    T.acc_g = (float*)(ws + lw.acc);
+    T.slots = (float*)(ws + lw.slots);
+    T.rec_floats = lw.rec_floats;
+    // Degrees of the fused kernel's two epilogue groups, balanced by rotate-back work
+    // ((2l + 1) per kept row: one m = 0 row and two per 0 < b <= min(l, mmax)); group 0
+    // starts with a share for the attention logits it also forms.
+    double work[8] = {0}, total = 0;
+    for (int l = 0; l <= desc->lmax; ++l) {
+      const int ml = l < desc->mmax ? l : desc->mmax;
+      work[l] = (2.0 * l + 1) * (1 + 2 * ml);
+      total += work[l];
+    }
+    double load[2] = {0.15 * total, 0.0};
+    bool done[8] = {false};
+    T.own_b = 0;
+    for (int it = 0; it <= desc->lmax; ++it) {
+      int best = -1;
+      for (int l = 0; l <= desc->lmax; ++l)
+        if (!done[l] && (best < 0 || work[l] > work[best])) best = l;
+      done[best] = true;
+      const int gsel = load[1] < load[0] ? 1 : 0;
+      load[gsel] += work[best];
+      if (gsel) T.own_b |= 1 << best;
+    }
+  } else {
+    T.wprep = ws + wl.wprep;
+    T.gates = (__nv_bfloat16*)(ws + wl.gate);
+    T.X = ws + wl.x;
+    T.Y = ws + wl.y;
+    T.logits = (float*)(ws + wl.logits);
+    T.Af = (float*)(ws + wl.af);
+  }
   TW.W2 = (const __nv_bfloat16*)W.W2;
   TW.W0 = (const __nv_bfloat16*)W.W0;
   for (int m = 0; m < 2; ++m)
@@ -362,7 +423,8 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
     case EGNN_WS_BUILD_GRAPH:
       return egnn_graph_workspace_bytes(n_atoms);
     case EGNN_WS_LAYER:
-      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc)) return tc_workspace(desc, n_edges, n_atoms).total;
+      if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
+        return layer_workspace(desc, n_edges, n_atoms).total;
       return 256;
     case EGNN_WS_HAMILTONIAN:
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
@@ -380,10 +442,18 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
   egnn_status s = check_desc(desc);
   if (s != EGNN_OK) return s;
   if ((s = check_graph(g, desc)) != EGNN_OK) return s;
-  if (!weights || !node_in || !node_out || node_in == node_out) return EGNN_ERR_INVALID_ARG;
+  if (!weights || !node_in || !node_out) return EGNN_ERR_INVALID_ARG;
+  {
+    // the aggregation reads neighbours' rows of node_in while other CTAs write node_out:
+    // the two byte ranges must be disjoint
+    const size_t bytes = (size_t)g->n_atoms * (desc->lmax + 1) * (desc->lmax + 1) * desc->channels *
+                         dtype_size(desc->dtype);
+    const uintptr_t a = (uintptr_t)node_in, b = (uintptr_t)node_out;
+    if (a < b + bytes && b < a + bytes) return EGNN_ERR_INVALID_ARG;
+  }
   cudaStream_t st = (cudaStream_t)cuda_stream;
   if (tc_eligible(desc)) {
-    TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
+    const LayerWorkspace wl = layer_workspace(desc, g->n_edges, g->n_atoms);
     if (!workspace || ws_bytes < wl.total) return EGNN_ERR_INVALID_ARG;
     if (((uintptr_t)weights | (uintptr_t)node_in | (uintptr_t)node_out) & 15) return EGNN_ERR_INVALID_ARG;
     uint8_t* ws = align1024(workspace);
@@ -391,8 +461,8 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
     carve_so2(W, (const char*)weights, desc, true);
     TcParams T;
     TcWeights TW;
-    fill_tc(T, TW, g, desc, W, node_in, node_out, ws, 1);
-    EGNN_CUDA_TRY(launch_layer_tc(T, TW, st));
+    fill_tc(T, TW, g, desc, W, node_in, node_out, ws, 1, nullptr, true);
+    EGNN_CUDA_TRY(launch_layer_fused(T, TW, st));
     return EGNN_OK;
   }
   So2Params P;
@@ -511,6 +581,12 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
   if (g->n_edges == 0) return EGNN_OK;
   EGNN_CUDA_TRY(launch_head_simt(P, W, T, st));
   // the tables live in `workspace`: keep them until the kernel has read them
+  return EGNN_OK;
+}
+
+extern "C" egnn_status egnn_check_bounded_wait(egnn_graph* g, uint32_t limit_us, void* cuda_stream) {
+  if (!g || !g->status || limit_us == 0 || limit_us > 2000000u) return EGNN_ERR_INVALID_ARG;
+  EGNN_CUDA_TRY(launch_wait_check(g->status, 1000ull * limit_us, (cudaStream_t)cuda_stream));
   return EGNN_OK;
 }
 

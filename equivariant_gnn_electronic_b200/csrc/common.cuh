@@ -6,17 +6,9 @@
 
 #include "egnn.h"
 
-// Device status codes written into egnn_graph::status (first writer wins).
-enum : int32_t {
-  EGNN_DEV_OK = 0,
-  EGNN_DEV_BAD_POSITION = 1,      // coordinate outside [0, box) or not finite
-  EGNN_DEV_SEGMENT_TOO_LARGE = 2, // more than the per-atom edge limit
-  EGNN_DEV_INDEX_RANGE = 3,       // a source index outside [0, n_atoms)
-  EGNN_DEV_COUNT_MISMATCH = 4,    // fill pass disagreed with count pass
-  EGNN_DEV_EDGE_OVERFLOW = 5,     // more than 2^31-1 edges
-  EGNN_DEV_WAIT_TIMEOUT = 6,      // a bounded wait in a pipelined kernel ran out
-  EGNN_DEV_BAD_GRAPH = 7          // row_ptr not monotone / out of range
-};
+// Device status codes written into egnn_graph::status (first writer wins): the
+// EGNN_DEV_* values of egnn.h.
+enum : int32_t { EGNN_DEV_OK = 0 };
 
 __device__ __forceinline__ void egnn_flag(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);

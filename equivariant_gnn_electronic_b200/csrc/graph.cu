@@ -419,6 +419,26 @@ extern "C" egnn_status egnn_build_graph(const double* pos, const int32_t* specie
   return EGNN_OK;
 }
 
+extern "C" egnn_status egnn_edge_geometry(const double* pos, const double box[3], egnn_graph* g,
+                                          void* cuda_stream) {
+  if (!pos || !box || !g || !g->row_ptr || !g->status || g->n_atoms < 1) return EGNN_ERR_INVALID_ARG;
+  if (g->n_edges < 0 || g->n_edges > g->capacity || g->n_edges > 0x7fffffffLL) return EGNN_ERR_INVALID_ARG;
+  if (g->n_edges > 0 && (!g->src || !g->shift || !g->dist || !g->wigner)) return EGNN_ERR_INVALID_ARG;
+  if (g->lmax < 0 || g->lmax > kLmaxW || g->mmax < 0 || g->mmax > 2 || g->mmax > g->lmax)
+    return EGNN_ERR_UNSUPPORTED;
+  for (int k = 0; k < 3; ++k)
+    if (!(box[k] > 0.0) || !(box[k] < 1e12)) return EGNN_ERR_INVALID_ARG;
+  if (g->n_edges == 0) return EGNN_OK;
+  cudaStream_t st = (cudaStream_t)cuda_stream;
+  const long long E = g->n_edges;
+  wigner_kernel<<<(int)((E + 127) / 128), 128, 0, st>>>(pos, g->n_atoms, g->row_ptr, g->src, g->shift, E, box[0],
+                                                         box[1], box[2], g->lmax, g->mmax,
+                                                         egnn_wigner_floats(g->lmax, g->mmax), g->dist, g->wigner,
+                                                         g->status);
+  EGNN_CUDA_TRY(cudaGetLastError());
+  return EGNN_OK;
+}
+
 // ---------------------------------------------------------------------------
 // egnn_build_graph_noalloc: the same graph build for callers that cannot hand the
 // library a device workspace.  Its scratch is a fixed array in this module's

@@ -11,15 +11,14 @@
 // here the contractions that are GEMMs run on tcgen05 and the small per-edge
 // rotations stay on the CUDA cores that feed them.
 //
-// Launches per layer (C = 128, bf16 storage, fp16 operands, fp32 accumulation):
+// Launches per layer (C = 128, bf16 storage and MMA operands, fp32 accumulation):
 //   prep_weights  packs the gate and SO(2) weight matrices into the exact
 //                 shared-memory image of K-major 128-byte-swizzled B tiles, one
 //                 tile per (pass, 64-wide K chunk), so one 1-D bulk copy moves it
 //                 (head: the label maps U^L are folded into the SO(2) rows here);
-//   to_f16        exact fp16 copy of the node table for the rotation.
 //   Then per range of at most 4096 edge tiles (128 edges each):
 //   gate          g_e = W2 SiLU(W1 rho(|r_e|) + b1) + b2 on tcgen05 (hidden layer on
-//                 the CUDA cores), fp16 per edge;
+//                 the CUDA cores), bf16 per edge;
 //   rotate        x_e = g_e * (D^l(R_e) [n_s || n_d]) for the kept rows |m| <= mmax,
 //                 written as ready-made A tiles;
 //   so2_gemm      D[128 x N <= 256] = A[128 x K] B[N x K]^T per pass in one of two
@@ -41,8 +40,8 @@
 namespace {
 
 constexpr int kSB = 2;                 // gate kernel B stages
-constexpr int kAStage = 128 * 128;     // one 128 x 64 fp16 A tile (16 KB)
-constexpr int kBStage = 256 * 128;     // one <= 256 x 64 fp16 B tile (32 KB)
+constexpr int kAStage = 128 * 128;     // one 128 x 64 bf16 A tile (16 KB)
+constexpr int kBStage = 256 * 128;     // one <= 256 x 64 bf16 B tile (32 KB)
 constexpr int kTmemCols = 512;
 constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = C = 128: two A tiles
 constexpr int kPW = 8;                 // gate kernel: warps computing the hidden layer
@@ -56,24 +55,8 @@ struct GateCtl {
   int abort;
 };
 
-__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ uint32_t pack2h(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
+using tc::pack2;
+using tc::unpack8;
 
 // Epilogue store of one 32-column group of a pass, cooperative over a warp that owns
 // 32 consecutive TMEM lanes (rows).  Each thread stages its row's 32 values in the
@@ -81,7 +64,7 @@ __device__ __forceinline__ uint32_t pack2h(float a, float b) {
 // both the row-wise writes and the column-wise reads); the warp then writes 4 rows
 // per instruction, each row's 32 columns contiguous, so every store covers whole
 // 128-byte (fp32) or 64-byte (16-bit) segments instead of 32 scattered pieces.
-// Gate passes add b2 and write fp16 gates; SO(2) passes write y (y0 in fp32, the
+// Gate passes add b2 and write bf16 gates; SO(2) passes write y (y0 in fp32, the
 // |m| > 0 blocks in bf16) or, in label mode, the fp32 label record.
 constexpr int kStageFloats = 32 * 36;   // per warp
 __device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& ps, float* st, long long e0,
@@ -126,8 +109,8 @@ __device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& 
     const int rr = r0 + rs;
     const float4 x = *reinterpret_cast<const float4*>(st + rr * 36 + c4);
     if (ps.kind == 0) {
-      __half* dst = P.gates + (grow0 + rr) * P.gcols + col + c4;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack2h(x.x, x.y), pack2h(x.z, x.w));
+      __nv_bfloat16* dst = P.gates + (grow0 + rr) * P.gcols + col + c4;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
     } else {
       const long long e = e0 + rr;
       if (e < P.n_edges) {
@@ -150,10 +133,10 @@ __device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& 
 
 // Radial gate GEMM, persistent over the tiles of a range: per 128-edge tile the
 // hidden layer h = SiLU(W1 rho(|r_e|) + b1) (K Gaussians) is computed on the CUDA
-// cores from W1 staged in shared memory and written as two 128 x 64 fp16 A tiles; the
+// cores from W1 staged in shared memory and written as two 128 x 64 bf16 A tiles; the
 // gate passes g = h W2^T (+ b2 in the epilogue) run on tcgen05 into two 256-column
 // TMEM accumulators used alternately, so one pass drains while the next accumulates.
-// Gates are written per edge in fp16.  Warp 0 bulk-copies W2 tiles, warp 1 issues
+// Gates are written per edge in bf16.  Warp 0 bulk-copies W2 tiles, warp 1 issues
 // the MMAs and owns TMEM, warps 2-9 compute the hidden layer (8 lanes per 128-byte row
 // slice, 4 rows per thread), warps 10-13 drain (thread = TMEM lane = edge).
 __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant__ TcParams P) {
@@ -247,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t ad = tc::sw128_desc(H_u32 + hb * kHStage + j * kAStage + ks * 32);
               const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
-              tc::mma_bf16(tmem + buf * 256, ad, bd, tc::idesc_f16(128, ps.n), (j > 0 || ks > 0) ? 1u : 0u);
+              tc::mma_bf16(tmem + buf * 256, ad, bd, tc::idesc_bf16(128, ps.n), (j > 0 || ks > 0) ? 1u : 0u);
             }
             tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
           }
@@ -319,10 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint4 w;
-          w.x = pack2h(v[j][0], v[j][1]);
-          w.y = pack2h(v[j][2], v[j][3]);
-          w.z = pack2h(v[j][4], v[j][5]);
-          w.w = pack2h(v[j][6], v[j][7]);
+          w.x = pack2(v[j][0], v[j][1]);
+          w.y = pack2(v[j][2], v[j][3]);
+          w.z = pack2(v[j][4], v[j][5]);
+          w.w = pack2(v[j][6], v[j][7]);
           *reinterpret_cast<uint4*>(Hb + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
         }
       }
@@ -426,7 +409,8 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
     const int o = ps.n_off + (r < ps.np ? r : r - ps.np);
     v = __bfloat162float(W[(long long)o * (nb * C2) + j * 64 + k]);
   }
-  reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);   // bf16 values are exact in fp16; label rows round once
+  // bf16 weights are copied exactly; label rows (U^L folded in, fp32 sums) round once
+  reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
 // Compile-time layout of kept row r = (l, m) (rows ordered by l, then m = -min(l,MM)..):
@@ -871,9 +855,10 @@ __global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcP
 // ---------------- rotate + gate: the A operands of the SO(2) GEMM ----------------
 // One CTA per 128-edge tile.  For every edge and degree l the kept rows of the edge
 // frame, x[l, m, :] = g[l, :] * sum_{m'} D^l[m, m'] [n_s || n_d][l, m', :] for
-// |m| <= min(l, mmax), are computed with packed fp16 FMAs from the fp16 copy of the
-// node table and written straight into the 128-byte-swizzled K-major 128 x 64 tiles
-// that the GEMM's bulk copies move (16-byte piece c of row r at position c ^ (r & 7)).
+// |m| <= min(l, mmax), are accumulated in fp32 (packed two-wide FMAs) from the bf16
+// node table, multiplied by the gates in fp32 and rounded once to the bf16 MMA operand,
+// then written straight into the 128-byte-swizzled K-major 128 x 64 tiles that the
+// GEMM's bulk copies move (16-byte piece c of row r at position c ^ (r & 7)).
 // Warp = one edge at a time, lane = one 8-channel piece of the 256-wide pair row
 // (lanes 0-15 the source atom, 16-31 the destination): a node row is one 512-byte
 // warp load, an A row four full 128-byte lines.  All 2l+1 rows of n[l] are loaded
@@ -911,61 +896,399 @@ __global__ void __launch_bounds__(256) rotate_kernel(const __grid_constant__ TcP
   for (int r = warp; r < 128; r += 8) {
     const long long e = (long long)t * 128 + r;
     const bool valid = e < E;
-    const __half* zn = P.node_h + (long long)s_node[side][r] * (L * L) * 128 + (lane & 15) * 8;
+    const __nv_bfloat16* zn = P.node_in + (long long)s_node[side][r] * (L * L) * 128 + (lane & 15) * 8;
     const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl;
-    const __half* gr = P.gates + ((long long)blockIdx.x * 128 + r) * P.gcols + lane * 8;
+    const __nv_bfloat16* gr = P.gates + ((long long)blockIdx.x * 128 + r) * P.gcols + lane * 8;
     uint8_t* xr = xt + r * 128 + ((qq ^ (r & 7)) << 4);
     int wo = 0;
 #pragma unroll
     for (int l = 0; l < L; ++l) {
       const int dl = 2 * l + 1, ml = l < MM ? l : MM, nr = 2 * ml + 1;
-      // the nr x dl kept coefficients of D^l, spread over the lanes as fp16 pairs
-      uint32_t cf[3];
+      // the nr x dl kept coefficients of D^l, spread over the lanes
+      float cf[3];
 #pragma unroll
       for (int k = 0; k < 3; ++k) {
         const int idx = lane + 32 * k;
-        const float v = (valid && idx < nr * dl) ? __ldg(De + wo + idx) : 0.f;
-        const __half2 h = __float2half2_rn(v);
-        cf[k] = *reinterpret_cast<const uint32_t*>(&h);
+        cf[k] = (valid && idx < nr * dl) ? __ldg(De + wo + idx) : 0.f;
       }
       uint4 zq[2 * LM + 1];
 #pragma unroll
       for (int mp = 0; mp < dl; ++mp)
         zq[mp] = valid ? __ldg(reinterpret_cast<const uint4*>(zn + (l * l + mp) * 128)) : make_uint4(0, 0, 0, 0);
       const uint4 gq = valid ? __ldg(reinterpret_cast<const uint4*>(gr + l * 256)) : make_uint4(0, 0, 0, 0);
-      __half2 acc[2 * MM + 1][4];
+      float2 acc[2 * MM + 1][4];
 #pragma unroll
       for (int m = 0; m < nr; ++m)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][i] = __float2half2_rn(0.f);
+        for (int i = 0; i < 4; ++i) acc[m][i] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int mp = 0; mp < dl; ++mp) {
-        const __half2* zh = reinterpret_cast<const __half2*>(&zq[mp]);
+        float z[8];
+        unpack8(zq[mp], z);
 #pragma unroll
         for (int m = 0; m < nr; ++m) {
           const int k = m * dl + mp;
-          const uint32_t cu = __shfl_sync(0xffffffffu, cf[k >> 5], k & 31);
-          const __half2 c = *reinterpret_cast<const __half2*>(&cu);
+          const float c = __shfl_sync(0xffffffffu, cf[k >> 5], k & 31);
+          const float2 c2 = make_float2(c, c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) acc[m][i] = __hfma2(c, zh[i], acc[m][i]);
+          for (int i = 0; i < 4; ++i) acc[m][i] = __ffma2_rn(c2, make_float2(z[2 * i], z[2 * i + 1]), acc[m][i]);
         }
       }
-      const __half2* gh = reinterpret_cast<const __half2*>(&gq);
+      float g[8];
+      unpack8(gq, g);
 #pragma unroll
       for (int m = 0; m < nr; ++m) {
         const int mm = m - ml, b = mm < 0 ? -mm : mm;
         const int id = b == 0 ? l * 4 + cs : P.xbase[b] + ((l - b) * 4 + cs) * 2 + (mm < 0 ? 1 : 0);
         uint4 w;
-        uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __half2 x = __hmul2(acc[m][i], gh[i]);
-          pw[i] = *reinterpret_cast<const uint32_t*>(&x);
-        }
+        w.x = pack2(acc[m][0].x * g[0], acc[m][0].y * g[1]);
+        w.y = pack2(acc[m][1].x * g[2], acc[m][1].y * g[3]);
+        w.z = pack2(acc[m][2].x * g[4], acc[m][2].y * g[5]);
+        w.w = pack2(acc[m][3].x * g[6], acc[m][3].y * g[7]);
         *reinterpret_cast<uint4*>(xr + (long long)id * 16384) = w;
       }
       wo += nr * dl;
     }
+  }
+}
+
+// ---------------- gate + rotate in one kernel: the A operands, gates kept on chip ----------------
+// Persistent over the tiles of a range (one CTA per SM).  Per 128-edge tile:
+//   rotation warps   the hidden layer h = SiLU(W1 rho(|r_e|) + b1) on the CUDA cores
+//                    (W1 staged in shared memory), written as the bf16 A operand of the
+//                    gate GEMM;
+//   MMA warp         per degree l one gate pass g[l] = h W2[l]^T (N = 2C = 256, K = C)
+//                    into one of two alternating 256-column TMEM accumulators;
+//   drain warps      thread = TMEM lane = edge: + b2, bf16, into one of two gate buffers
+//                    G[edge][256] in shared memory (16-byte piece j of row r at j ^ (r & 31));
+//   rotation warps   x_e[l, m, :] = g_e[l, :] * sum_{m'} D^l_e[m, m'] [n_s || n_d][l, m', :]
+//                    for |m| <= min(l, mmax): fp32 accumulation, one rounding to bf16, into
+//                    the 128-byte-swizzled K-major A tiles the SO(2) layer reads (warp = one
+//                    edge at a time, lane = 8 of the 256 pair channels).
+// The gates never leave the SM; degree l + 1 is gated while degree l is rotated.
+constexpr int kGRB = 3;                        // W2 tile stages (128 rows x 64 K, 16 KB)
+constexpr int kGRRot = 8;                      // hidden-layer / rotation warps
+constexpr int kGRThreads = (2 + 4 + kGRRot) * 32;
+constexpr int kGRTile = 128 * 128;             // one 128 x 64 bf16 tile
+constexpr int kGBuf = 128 * 512;               // gates of one degree: 128 edges x 256 bf16
+constexpr uint32_t kRotBar = 2;                // named barrier of the rotation warps
+
+struct GRCtl {
+  uint64_t b_full[kGRB], b_empty[kGRB], acc_full[2], acc_empty[2];
+  uint64_t hid_full, hid_empty, g_full[2], g_empty[2], mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int node[2][128];                            // source and destination atom of each row
+};
+
+size_t gate_rotate_smem_bytes(int K, int C) {
+  return kGRB * kGRTile + 2 * kGRTile + 2 * kGBuf + (size_t)K * C * 2 + sizeof(GRCtl) + 1024;
+}
+
+template <int LM, int MM>
+__global__ void __launch_bounds__(kGRThreads, 1) gate_rotate_kernel(const __grid_constant__ TcParams P) {
+  constexpr int L = LM + 1;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = tc::smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const uint32_t B_u32 = base_u32;
+  uint8_t* Hbuf = base + kGRB * kGRTile;
+  const uint32_t H_u32 = B_u32 + kGRB * kGRTile;
+  uint8_t* Gbuf = Hbuf + 2 * kGRTile;
+  __nv_bfloat16* W1s = reinterpret_cast<__nv_bfloat16*>(Gbuf + 2 * kGBuf);   // [K][C]
+  GRCtl* ctl = reinterpret_cast<GRCtl*>(reinterpret_cast<uint8_t*>(W1s) + (((size_t)P.K * P.C * 2 + 15) & ~15));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &ctl->abort;
+  const int C = P.C, K = P.K;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGRB; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->b_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->b_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(tc::smem_u32(&ctl->acc_full[i]), 1);
+      tc::mbar_init(tc::smem_u32(&ctl->acc_empty[i]), 128);
+      tc::mbar_init(tc::smem_u32(&ctl->g_full[i]), 128);
+      tc::mbar_init(tc::smem_u32(&ctl->g_empty[i]), kGRRot * 32);
+    }
+    tc::mbar_init(tc::smem_u32(&ctl->hid_full), kGRRot * 32);
+    tc::mbar_init(tc::smem_u32(&ctl->hid_empty), 1);
+    tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
+    ctl->abort = 0;
+    tc::fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < C * K; i += blockDim.x) {
+    const int c = i / K, k = i - c * K;
+    W1s[k * C + c] = P.W1[i];
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(&ctl->tmem_base), 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const long long E = P.n_edges;
+
+  if (warp == 0) {
+    // ---------------- W2 tiles: per degree, two K chunks x two 128-row halves ----------------
+    if (lane == 0) {
+      uint32_t ib = 0;
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
+        for (int l = 0; l < L && !*abort; ++l) {
+          for (int j = 0; j < 4 && !*abort; ++j, ++ib) {
+            const int sb = ib % kGRB;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kGRB) & 1) ^ 1, P.status, abort, 64)) break;
+            tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->b_full[sb]), (uint32_t)kGRTile);
+            tc::bulk_g2s(B_u32 + sb * kGRTile, P.wprep + P.pass[l].boff + (long long)j * kGRTile,
+                         (uint32_t)kGRTile, tc::smem_u32(&ctl->b_full[sb]));
+          }
+        }
+      }
+      for (uint32_t k = (ib > (uint32_t)kGRB ? ib - kGRB : 0); k < ib; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kGRB]);
+        const uint64_t t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(bar, (k / kGRB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- gate MMAs: D[edges][256 gates of degree l] = h W2[l]^T ----------------
+    if (lane == 0) {
+      const uint32_t id = tc::idesc_bf16(128, 128);
+      uint32_t ib = 0, it = 0, ig = 0;
+      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full), it & 1, P.status, abort, 32)) break;
+        for (int l = 0; l < L && !*abort; ++l, ++ig) {
+          const int ab = ig & 1;
+          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty[ab]), ((ig >> 1) & 1) ^ 1, P.status, abort, 32)) break;
+          tc::tc_fence_after();
+          for (int kc = 0; kc < 2; ++kc, ib += 2) {
+            const int s0 = ib % kGRB, s1 = (ib + 1) % kGRB;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[s0]), (ib / kGRB) & 1, P.status, abort)) break;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[s1]), ((ib + 1) / kGRB) & 1, P.status, abort)) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = tc::sw128_desc(H_u32 + kc * kGRTile + ks * 32);
+              const uint32_t a = (kc > 0 || ks > 0) ? 1u : 0u;
+              tc::mma_bf16(tmem + ab * 256, ad, tc::sw128_desc(B_u32 + s0 * kGRTile + ks * 32), id, a);
+              tc::mma_bf16(tmem + ab * 256 + 128, ad, tc::sw128_desc(B_u32 + s1 * kGRTile + ks * 32), id, a);
+            }
+            tc::mma_commit(tc::smem_u32(&ctl->b_empty[s0]));
+            tc::mma_commit(tc::smem_u32(&ctl->b_empty[s1]));
+          }
+          tc::mma_commit(tc::smem_u32(&ctl->acc_full[ab]));
+        }
+        tc::mma_commit(tc::smem_u32(&ctl->hid_empty));
+      }
+      tc::mma_commit(tc::smem_u32(&ctl->mma_done));
+      const uint64_t t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(tc::smem_u32(&ctl->mma_done), 0) && tc::globaltimer() - t0 < 2000000000ull) {
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---------------- drain: thread = TMEM lane = edge; + b2, bf16, into G ----------------
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    uint32_t ig = 0;
+    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
+      for (int l = 0; l < L; ++l, ++ig) {
+        const int ab = ig & 1;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[ab]), (ig >> 1) & 1, P.status, abort, 64)) break;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->g_empty[ab]), ((ig >> 1) & 1) ^ 1, P.status, abort, 64)) break;
+        tc::tc_fence_after();
+        uint8_t* grow = Gbuf + ab * kGBuf + r * 512;
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+          uint32_t y[32];
+          tc::tmem_ld32_issue(tl + ab * 256 + 32 * j, y);
+          tc::tmem_ld_wait(y);
+          const uint4* bp = reinterpret_cast<const uint4*>(P.b2 + l * 256 + 32 * j);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float bv[8];
+            tc::unpack8(__ldg(bp + u), bv);
+            uint4 w;
+            w.x = pack2(__uint_as_float(y[8 * u]) + bv[0], __uint_as_float(y[8 * u + 1]) + bv[1]);
+            w.y = pack2(__uint_as_float(y[8 * u + 2]) + bv[2], __uint_as_float(y[8 * u + 3]) + bv[3]);
+            w.z = pack2(__uint_as_float(y[8 * u + 4]) + bv[4], __uint_as_float(y[8 * u + 5]) + bv[5]);
+            w.w = pack2(__uint_as_float(y[8 * u + 6]) + bv[6], __uint_as_float(y[8 * u + 7]) + bv[7]);
+            *reinterpret_cast<uint4*>(grow + (((4 * j + u) ^ (r & 31)) << 4)) = w;
+          }
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[ab]));
+        tc::mbar_arrive(tc::smem_u32(&ctl->g_full[ab]));
+      }
+    }
+  } else {
+    // ---------------- hidden layer and rotation ----------------
+    // Waits here ignore the abort flag (they time out on their own) so that every
+    // rotation thread leaves at the same point and none is left at the named barrier.
+    volatile int no_abort = 0;
+    const int rw = warp - 6, rt = threadIdx.x - 6 * 32;
+    const int side = lane >> 4, cs = lane >> 3, qq = lane & 7;
+    const int pq = rt & 7, prb = rt >> 3;           // hidden layer: 16-byte piece, row group
+    const float mu_step = P.rcut / (float)(K - 1);
+    const float inv2s2 = 1.0f / (2.0f * mu_step * mu_step);
+    float b1v[2][8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b1v[j][i] = __bfloat162float(P.b1[j * 64 + pq * 8 + i]);
+    uint32_t it = 0, ig = 0;
+    bool failed = false;
+    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !failed; t += gridDim.x, ++it) {
+      tc::bar_sync(kRotBar, kGRRot * 32);   // the previous tile's rows are done with ctl->node
+      if (rt < 128) {
+        const long long e = (long long)t * 128 + rt;
+        int sv = 0, dv = 0;
+        if (e < E) {
+          sv = P.src[e];
+          int lo = 0, hi = P.n_atoms;
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+          }
+          dv = lo;
+          if (sv < 0 || sv >= P.n_atoms) {
+            egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
+            sv = dv;
+          }
+        }
+        ctl->node[0][rt] = sv;
+        ctl->node[1][rt] = dv;
+      }
+      // hidden layer of the tile (the gate MMAs of the previous tile are done with H)
+      if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty), (it & 1) ^ 1, P.status, &no_abort, 64)) {
+        failed = true;
+        break;
+      }
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int r = prb + 32 * u;
+        const long long e = (long long)t * 128 + r;
+        float v[2][8];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[j][i] = 0.f;
+        if (e < E) {
+          const float di = P.dist[e];
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[j][i] = b1v[j][i];
+          for (int k = 0; k < K; ++k) {
+            const float dd = di - k * mu_step;
+            const float rho = __expf(-dd * dd * inv2s2);
+            const uint4* w = reinterpret_cast<const uint4*>(W1s + k * C + pq * 8);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              float wv[8];
+              tc::unpack8(w[j * 8], wv);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[j][i] = fmaf(wv[i], rho, v[j][i]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[j][i] = __fdividef(v[j][i], 1.0f + __expf(-v[j][i]));
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint4 w;
+          w.x = pack2(v[j][0], v[j][1]);
+          w.y = pack2(v[j][2], v[j][3]);
+          w.z = pack2(v[j][4], v[j][5]);
+          w.w = pack2(v[j][6], v[j][7]);
+          *reinterpret_cast<uint4*>(Hbuf + j * kGRTile + r * 128 + ((pq ^ (r & 7)) << 4)) = w;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(tc::smem_u32(&ctl->hid_full));
+      tc::bar_sync(kRotBar, kGRRot * 32);   // ctl->node of this tile is complete
+      uint8_t* xt = P.X + (long long)(t - P.t_begin) * P.nch * 16384;
+      int wo = 0;
+#pragma unroll
+      for (int l = 0; l < L; ++l, ++ig) {
+        const int gb = ig & 1;
+        const int dl = 2 * l + 1, ml = l < MM ? l : MM, nr = 2 * ml + 1;
+        if (!tc::mbar_wait(tc::smem_u32(&ctl->g_full[gb]), (ig >> 1) & 1, P.status, &no_abort, 64)) {
+          failed = true;
+          break;
+        }
+        const uint8_t* G = Gbuf + gb * kGBuf;
+        for (int r = rw; r < 128; r += kGRRot) {
+          const long long e = (long long)t * 128 + r;
+          const bool valid = e < E;
+          const __nv_bfloat16* zn =
+              P.node_in + ((long long)ctl->node[side][r] * (L * L) + l * l) * 128 + (lane & 15) * 8;
+          const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl + wo;
+          float cf[3];
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            const int idx = lane + 32 * k;
+            cf[k] = (valid && idx < nr * dl) ? __ldg(De + idx) : 0.f;
+          }
+          uint4 zq[2 * LM + 1];
+#pragma unroll
+          for (int mp = 0; mp < dl; ++mp)
+            zq[mp] = valid ? __ldg(reinterpret_cast<const uint4*>(zn + mp * 128)) : make_uint4(0, 0, 0, 0);
+          const uint4 gq = *reinterpret_cast<const uint4*>(G + r * 512 + ((lane ^ (r & 31)) << 4));
+          float2 acc[2 * MM + 1][4];
+#pragma unroll
+          for (int m = 0; m < nr; ++m)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[m][i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int mp = 0; mp < dl; ++mp) {
+            float z[8];
+            unpack8(zq[mp], z);
+#pragma unroll
+            for (int m = 0; m < nr; ++m) {
+              const int k = m * dl + mp;
+              const float cv = __shfl_sync(0xffffffffu, cf[k >> 5], k & 31);
+              const float2 c2 = make_float2(cv, cv);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc[m][i] = __ffma2_rn(c2, make_float2(z[2 * i], z[2 * i + 1]), acc[m][i]);
+            }
+          }
+          float g[8];
+          unpack8(gq, g);
+          uint8_t* xr = xt + r * 128 + ((qq ^ (r & 7)) << 4);
+#pragma unroll
+          for (int m = 0; m < nr; ++m) {
+            const int mm = m - ml, b = mm < 0 ? -mm : mm;
+            const int id = b == 0 ? l * 4 + cs : P.xbase[b] + ((l - b) * 4 + cs) * 2 + (mm < 0 ? 1 : 0);
+            uint4 w;
+            w.x = pack2(acc[m][0].x * g[0], acc[m][0].y * g[1]);
+            w.y = pack2(acc[m][1].x * g[2], acc[m][1].y * g[3]);
+            w.z = pack2(acc[m][2].x * g[4], acc[m][2].y * g[5]);
+            w.w = pack2(acc[m][3].x * g[6], acc[m][3].y * g[7]);
+            *reinterpret_cast<uint4*>(xr + (long long)id * 16384) = w;
+          }
+        }
+        tc::mbar_arrive(tc::smem_u32(&ctl->g_empty[gb]));
+        wo += nr * dl;
+      }
+    }
+    if (failed) {
+      egnn_flag(P.status, EGNN_DEV_WAIT_TIMEOUT);
+      *abort = 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -976,7 +1299,7 @@ __global__ void __launch_bounds__(256) rotate_kernel(const __grid_constant__ TcP
 constexpr int kNBuf = kTcAccCols == 256 ? 2 : 1;    // TMEM accumulators
 constexpr int kGA = kNBuf == 2 ? 6 : 4;              // A stages (16 KB each)
 constexpr int kGB = kNBuf == 2 ? 3 : 2;              // B stages
-constexpr int kGBStage = kTcAccCols * 128;           // one <= kTcAccCols x 64 fp16 B tile
+constexpr int kGBStage = kTcAccCols * 128;           // one <= kTcAccCols x 64 bf16 B tile
 constexpr int kGThreads = 6 * 32;
 
 struct GemmCtl {
@@ -1079,7 +1402,7 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
           if (ps.block > 0) {
             // y+ += x+ W1^T - x- W2^T ; y- += x+ W2^T + x- W1^T, one K block of 64 per step
             const int np = ps.np;
-            const uint32_t idn = tc::idesc_f16(128, np), idneg = tc::idesc_f16(128, np, true);
+            const uint32_t idn = tc::idesc_bf16(128, np), idneg = tc::idesc_bf16(128, np, true);
             for (int kb = 0; kb < ps.nk; ++kb, ++ib, ia += 2) {
               const int sb = ib % kGB, sp = ia % kGA, sm = (ia + 1) % kGA;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kGB) & 1, P.status, abort)) break;
@@ -1114,7 +1437,7 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
                 for (int n0 = 0; n0 < ps.n; n0 += 256) {
                   const int ns = ps.n - n0 < 256 ? ps.n - n0 : 256;
                   const uint64_t bd = tc::sw128_desc(B_u32 + sb * kGBStage + n0 * 128 + ks * 32);
-                  tc::mma_bf16(acc_t + n0, ad, bd, tc::idesc_f16(128, ns), (kb > 0 || ks > 0) ? 1u : 0u);
+                  tc::mma_bf16(acc_t + n0, ad, bd, tc::idesc_bf16(128, ns), (kb > 0 || ks > 0) ? 1u : 0u);
                 }
               }
               tc::mma_commit(tc::smem_u32(&ctl->a_empty[sa]));
@@ -1204,24 +1527,27 @@ size_t gate_smem_bytes(int K, int C) {
   return kSB * kBStage + 2 * kHStage + sizeof(float) * ((size_t)K * C + 4 * kStageFloats) + sizeof(GateCtl) + 1024;
 }
 
-// bf16 -> fp16 copy of the node table (exact for the embeddings' range), 8 values per thread.
-__global__ void to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half* __restrict__ out, long long n8) {
-  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const uint4 q = reinterpret_cast<const uint4*>(in)[i];
-  float f[8];
-  unpack8(q, f);
-  uint4 o;
-  o.x = pack2h(f[0], f[1]);
-  o.y = pack2h(f[2], f[3]);
-  o.z = pack2h(f[4], f[5]);
-  o.w = pack2h(f[6], f[7]);
-  reinterpret_cast<uint4*>(out)[i] = o;
-}
-
 __global__ void a_to_f32_kernel(const __nv_bfloat16* __restrict__ A, float* __restrict__ out, int n) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = __bfloat162float(A[i]);
+}
+
+// Check of the bounded wait every pipelined kernel uses: one thread waits on an
+// mbarrier that nothing arrives on, with the given limit, through the same routine
+// (tc::mbar_wait); when the limit runs out it records EGNN_DEV_WAIT_TIMEOUT in *status.
+__global__ void wait_check_kernel(int32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x != 0) return;
+  tc::mbar_init(tc::smem_u32(&bar), 1);
+  abort = 0;
+  tc::fence_barrier_init();
+  tc::mbar_wait(tc::smem_u32(&bar), 0, status, &abort, 0, limit_ns);
+}
+
+cudaError_t launch_wait_check(int32_t* status, unsigned long long limit_ns, cudaStream_t st) {
+  wait_check_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
 }
 
 // ---- opt-in timing of the SO(2) GEMM launches of layer calls (diagnostics) ----
@@ -1280,14 +1606,32 @@ static cudaError_t launch_rotate_any(const TcParams& P, int nt, cudaStream_t st)
   return cudaGetLastError();
 }
 
-// Weight prep, then per range of edge tiles: gate GEMM -> rotate -> SO(2) GEMM.
-static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStream_t st) {
-  if (P.with_logits) {
-    const int na = P.H * P.L * P.C;
-    a_to_f32_kernel<<<(na + 255) / 256, 256, 0, st>>>(P.A, P.Af, na);
+static cudaError_t launch_gate_rotate_any(const TcParams& P, int grid, size_t smem, cudaStream_t st) {
+  cudaError_t err = cudaSuccess;
+  switch (P.mmax * 8 + P.lmax) {
+#define EGNN_GR_CASE(LMv, MMv)                                                                           \
+  case MMv * 8 + LMv:                                                                                   \
+    err = cudaFuncSetAttribute(gate_rotate_kernel<LMv, MMv>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                               (int)smem);                                                              \
+    if (err != cudaSuccess) return err;                                                                 \
+    gate_rotate_kernel<LMv, MMv><<<grid, kGRThreads, smem, st>>>(P);                                     \
+    break;
+    EGNN_GR_CASE(1, 0) EGNN_GR_CASE(2, 0) EGNN_GR_CASE(3, 0) EGNN_GR_CASE(4, 0) EGNN_GR_CASE(5, 0)
+    EGNN_GR_CASE(6, 0) EGNN_GR_CASE(1, 1) EGNN_GR_CASE(2, 1) EGNN_GR_CASE(3, 1) EGNN_GR_CASE(4, 1)
+    EGNN_GR_CASE(5, 1) EGNN_GR_CASE(6, 1) EGNN_GR_CASE(2, 2) EGNN_GR_CASE(3, 2) EGNN_GR_CASE(4, 2)
+    EGNN_GR_CASE(5, 2) EGNN_GR_CASE(6, 2)
+#undef EGNN_GR_CASE
+    default:
+      return cudaErrorInvalidValue;
   }
-  const long long n8 = (long long)P.n_atoms * P.L2 * P.C / 8;
-  to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(P.node_in, P.node_h, n8);
+  return cudaGetLastError();
+}
+
+// Weight prep, then per range of edge tiles: gates + rotation (one kernel) -> the
+// consumer of the range's A tiles (the SO(2) GEMM of the head, or the fused layer kernel).  Each
+// consumer launch is bracketed by the opt-in profiling events when `profiled`.
+cudaError_t launch_tc_pipeline(const TcParams& P, const TcWeights& W, cudaStream_t st, TcConsumer consumer,
+                               void* ctx, bool profiled) {
   long long total = P.wprep_bytes / 2;
   prep_weights_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(P, W.W2, W.W0, W.Wm[0][0], W.Wm[0][1],
                                                                       W.Wm[1][0], W.Wm[1][1], total,
@@ -1301,14 +1645,7 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
   Pg.npass = ng;
   Ps.npass = P.npass - ng;
   for (int i = 0; i < Ps.npass; ++i) Ps.pass[i] = P.pass[ng + i];
-  const size_t sm_g = gate_smem_bytes(P.K, P.C);
-  const size_t sm_s = kGA * kAStage + kGB * kGBStage + sizeof(float) * 4 * kStageFloats + sizeof(GemmCtl) + 1024;
-  if ((err = cudaFuncSetAttribute(gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) !=
-      cudaSuccess)
-    return err;
-  if ((err = cudaFuncSetAttribute(so2_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_s)) !=
-      cudaSuccess)
-    return err;
+  const size_t sm_g = gate_rotate_smem_bytes(P.K, P.C);
   const int tch = tc_chunk_tiles(P.n_tiles);
   for (int tb = 0; tb < P.n_tiles; tb += tch) {
     const int te = tb + tch < P.n_tiles ? tb + tch : P.n_tiles;
@@ -1316,11 +1653,9 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
     const int grid = P.grid < nt ? P.grid : nt;
     Pg.t_begin = Ps.t_begin = tb;
     Pg.t_end = Ps.t_end = te;
-    gate_kernel<<<grid, kThreads, sm_g, st>>>(Pg);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if ((err = launch_rotate_any(Ps, nt, st)) != cudaSuccess) return err;
+    if ((err = launch_gate_rotate_any(Pg, grid, sm_g, st)) != cudaSuccess) return err;
     const int pi = g_prof_n;
-    const bool prof = g_prof_on && P.with_logits && !P.label_mode && pi < kProfMax;
+    const bool prof = profiled && g_prof_on && pi < kProfMax;
     if (prof) {
       if (!g_prof_made[pi]) {
         if ((err = cudaEventCreate(&g_prof_ev[0][pi])) != cudaSuccess) return err;
@@ -1329,8 +1664,7 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
       }
       if ((err = cudaEventRecord(g_prof_ev[0][pi], st)) != cudaSuccess) return err;
     }
-    so2_gemm_kernel<<<grid, kGThreads, sm_s, st>>>(Ps);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = consumer(Ps, grid, st, ctx)) != cudaSuccess) return err;
     if (prof) {
       if ((err = cudaEventRecord(g_prof_ev[1][pi], st)) != cudaSuccess) return err;
       const long long e_end = (long long)te * 128 < P.n_edges ? (long long)te * 128 : P.n_edges;
@@ -1339,6 +1673,22 @@ static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStr
     }
   }
   return cudaSuccess;
+}
+
+static cudaError_t so2_gemm_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*) {
+  const size_t sm_s = kGA * kAStage + kGB * kGBStage + sizeof(float) * 4 * kStageFloats + sizeof(GemmCtl) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(so2_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_s);
+  if (err != cudaSuccess) return err;
+  so2_gemm_kernel<<<grid, kGThreads, sm_s, st>>>(Ps);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStream_t st) {
+  if (P.with_logits) {
+    const int na = P.H * P.L * P.C;
+    a_to_f32_kernel<<<(na + 255) / 256, 256, 0, st>>>(P.A, P.Af, na);
+  }
+  return launch_tc_pipeline(P, W, st, so2_gemm_consumer, nullptr, P.with_logits && !P.label_mode);
 }
 
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te) {

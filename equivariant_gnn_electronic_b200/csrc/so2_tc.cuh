@@ -1,7 +1,6 @@
 // Launch parameters of the tensor-core eSCN layer (CUDA path only).
 #pragma once
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,7 +34,6 @@ struct TcParams {
   const float* wig;
   const __nv_bfloat16* node_in;
   __nv_bfloat16* node_out;
-  __half* node_h;                // fp16 copy of node_in (exact), read by the rotate kernel
   const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
   const uint8_t* wprep;
   long long wprep_bytes;
@@ -54,15 +52,26 @@ struct TcParams {
   int mult[8];                   // labels per L
   const __nv_bfloat16* U[8];     // U^L [mult_L][C]
   // Tile range of one launch and the per-range buffers of the split pipeline
-  // (gate GEMM -> rotate -> SO(2) GEMM): gates of the range's rows in fp16, and the
-  // rotated, gated A operands as 128 x 64 fp16 tiles in the 128-byte-swizzled
+  // (gate GEMM -> rotate -> SO(2) GEMM): gates of the range's rows in bf16, and the
+  // rotated, gated A operands as 128 x 64 bf16 tiles in the 128-byte-swizzled
   // K-major image the MMA reads, `nch` tiles per edge tile, block b's first at
   // xbase[b] (a |m| > 0 K block stores x+ then x-).
   int t_begin, t_end;
-  __half* gates;                 // [(t_end - t_begin) * 128][gcols]
+  __nv_bfloat16* gates;          // [(t_end - t_begin) * 128][gcols]
   uint8_t* X;                    // [(t_end - t_begin)][nch][128 * 128 B]
   int nch;
   int xbase[3];
+  // Fused layer (layer_fused_kernel): per-CTA stash of y0 in bf16, [grid][L][128][C];
+  // per-atom fp32 accumulators of the destinations whose incoming edges lie inside one
+  // edge tile, [n_atoms][L^2][C]; and two partial records per edge tile for the
+  // destinations whose edges cross a tile boundary, [n_tiles][2][rec_floats], a record
+  // being the unnormalised weighted sum [L^2][C], then the per-head softmax maximum [16]
+  // and denominator [16] of the tile's part of the segment.
+  __nv_bfloat16* stash;
+  float* acc_g;
+  float* slots;
+  int rec_floats;
+  int own_b;                     // bit l set: the fused layer's second epilogue group owns degree l
   int npass;
   TcPass pass[32];
   int woff[8];
@@ -103,9 +112,16 @@ struct HeadUPtrs {
 };
 
 size_t gate_smem_bytes(int K, int C);
+// Consumer of one range's A tiles: launches its kernel over tiles [Ps.t_begin, Ps.t_end).
+using TcConsumer = cudaError_t (*)(const TcParams& Ps, int grid, cudaStream_t st, void* ctx);
+cudaError_t launch_tc_pipeline(const TcParams& P, const TcWeights& W, cudaStream_t st, TcConsumer consumer,
+                               void* ctx, bool profiled);
 cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st);
+cudaError_t launch_layer_fused(const TcParams& P, const TcWeights& W, cudaStream_t st);
+size_t layer_fused_smem_bytes(int lmax, int heads);
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
                            float* blocks, cudaStream_t st);
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te);
 void tc_profile_enable(bool on);
+cudaError_t launch_wait_check(int32_t* status, unsigned long long limit_ns, cudaStream_t st);
 cudaError_t tc_profile_read(double* ms, long long* launches, long long* edges);

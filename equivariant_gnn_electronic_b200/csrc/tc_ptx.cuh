@@ -1,5 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, bulk copies, tcgen05 (CUDA path only).
 #pragma once
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -44,20 +45,21 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Bounded wait: gives up after ~2 s of wall time (or when *abort is set by another
-// role), records EGNN_DEV_WAIT_TIMEOUT and returns false.  Never traps.
+// Bounded wait: gives up after `limit_ns` of wall time (2 s by default) or when *abort
+// is set by another role, records EGNN_DEV_WAIT_TIMEOUT and returns false.  Never traps.
 // `sleep_ns` > 0 makes a waiting warp yield its issue slot between polls (roles that
 // wait long and are not latency-critical), so it does not steal issue bandwidth from
 // the warps doing the work on the same SM sub-partition.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status,
-                                          volatile int* abort, uint32_t sleep_ns = 0) {
+                                          volatile int* abort, uint32_t sleep_ns = 0,
+                                          uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   while (true) {
     if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > 2000000000ull) {
+    if (globaltimer() - t0 > limit_ns) {
       egnn_flag(status, EGNN_DEV_WAIT_TIMEOUT);
       *abort = 1;
       return false;
@@ -153,6 +155,22 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
                : "memory");
 }
 
+// 32 lanes x 8 consecutive 32-bit columns (issue only; complete with tmem_ld_wait8).
+__device__ __forceinline__ void tmem_ld8_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+// Waits for every tcgen05.ld of the thread; names two 8-register destinations so that no
+// use of them is scheduled before it.
+__device__ __forceinline__ void tmem_ld_wait8x2(uint32_t* a, uint32_t* b) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                 "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])
+               :
+               : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B,
 // 8-row groups 1024 B apart (SBO), LBO unused (1), version 1, layout type 2.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -165,9 +183,65 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M x N.
-__host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M x N; negate_b / negate_a
+// flip the sign of B / A.
+__host__ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N, bool negate_b = false,
+                                                        bool negate_a = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (negate_a ? (1u << 13) : 0u) | (negate_b ? (1u << 14) : 0u) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- CUDA-core helpers shared by the bf16 kernels ----
+// 8 bf16 (one 16-byte word) -> fp32: a bf16 is the high half of the fp32 with the same value.
+__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 4-byte asynchronous copy global -> shared (no registers held); complete with
+// cp_async_wait_all.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Named barrier over `count` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Fire-and-forget fp32 add to global memory (no value returned).  No memory clobber:
+// callers order it against their own accesses of the same address by program order
+// (one writing thread per address), and shared-memory loads may move across it.
+__device__ __forceinline__ void red_add(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v));
+}
+
+// Four 8x8 b16 matrices from shared memory; lane i supplies the address of row (i & 7)
+// of matrix (i >> 3).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// Warp-level D[16x8] += A[16x16] B[16x8], bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 // Instruction descriptor: f16 x f16 -> fp32, both K-major, M x N; negate_b flips B's sign.
 __host__ __device__ __forceinline__ uint32_t idesc_f16(int M, int N, bool negate_b = false) {

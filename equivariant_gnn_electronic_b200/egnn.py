@@ -23,8 +23,10 @@ EGNN_WS_BUILD_GRAPH, EGNN_WS_LAYER, EGNN_WS_HAMILTONIAN = 0, 1, 2
 EXPORTED = (
     "egnn_wigner_floats", "egnn_workspace_bytes", "egnn_build_graph", "egnn_layer_forward",
     "egnn_hamiltonian_blocks", "egnn_read_status", "egnn_status_string", "egnn_build_graph_noalloc",
-    "egnn_profile", "egnn_profile_read",
+    "egnn_profile", "egnn_profile_read", "egnn_edge_geometry", "egnn_check_bounded_wait",
 )
+EGNN_DEV_BAD_POSITION, EGNN_DEV_SEGMENT_TOO_LARGE, EGNN_DEV_INDEX_RANGE, EGNN_DEV_COUNT_MISMATCH, \
+    EGNN_DEV_EDGE_OVERFLOW, EGNN_DEV_WAIT_TIMEOUT, EGNN_DEV_BAD_GRAPH = range(1, 8)
 
 
 class LayerDesc(ctypes.Structure):
@@ -71,6 +73,10 @@ def _load():
     lib.egnn_read_status.restype = i32
     lib.egnn_status_string.argtypes = [i32]
     lib.egnn_status_string.restype = ctypes.c_char_p
+    lib.egnn_edge_geometry.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(GraphStruct), vp]
+    lib.egnn_edge_geometry.restype = i32
+    lib.egnn_check_bounded_wait.argtypes = [ctypes.POINTER(GraphStruct), ctypes.c_uint32, vp]
+    lib.egnn_check_bounded_wait.restype = i32
     lib.egnn_profile.argtypes = [i32]
     lib.egnn_profile.restype = i32
     lib.egnn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), ctypes.POINTER(i64)]
@@ -101,12 +107,12 @@ def _ptr(t: Optional[torch.Tensor]):
 
 
 def profile(enable: bool) -> None:
-    """Start (clearing the record) or stop timing the SO(2) GEMM launches of layer calls."""
+    """Start (clearing the record) or stop timing the fused-kernel launches of layer calls."""
     _check(lib.egnn_profile(1 if enable else 0), "egnn_profile")
 
 
 def profile_read() -> tuple[float, int, int]:
-    """(summed GEMM launch milliseconds, launches, edges processed) of the record."""
+    """(summed fused-kernel launch milliseconds, launches, edges processed) of the record."""
     ms, n, e = ctypes.c_double(0.0), ctypes.c_int64(0), ctypes.c_int64(0)
     _check(lib.egnn_profile_read(ctypes.byref(ms), ctypes.byref(n), ctypes.byref(e)), "egnn_profile_read")
     return ms.value, n.value, e.value
@@ -212,6 +218,20 @@ def build_graph_noalloc(pos: torch.Tensor, species: torch.Tensor, box: Sequence[
     boxarr = (ctypes.c_double * 3)(*[float(b) for b in box])
     return int(lib.egnn_build_graph_noalloc(_ptr(pos), _ptr(species), pos.shape[0], boxarr, float(rcut),
                                             lmax, mmax, ctypes.byref(graph.s), _stream(stream)))
+
+
+def edge_geometry(pos: torch.Tensor, box: Sequence[float], graph: Graph, stream=None) -> Graph:
+    """Distances and Wigner rows of graph's edges for new positions (same neighbour list)."""
+    assert pos.dtype == torch.float64 and pos.is_cuda and pos.is_contiguous()
+    boxarr = (ctypes.c_double * 3)(*[float(b) for b in box])
+    _check(lib.egnn_edge_geometry(_ptr(pos), boxarr, ctypes.byref(graph.s), _stream(stream)), "egnn_edge_geometry")
+    return graph
+
+
+def check_bounded_wait(graph: Graph, limit_us: int, stream=None) -> None:
+    """Run the pipelined kernels' bounded wait on an mbarrier nothing arrives on."""
+    _check(lib.egnn_check_bounded_wait(ctypes.byref(graph.s), int(limit_us), _stream(stream)),
+           "egnn_check_bounded_wait")
 
 
 def layer_forward(graph: Graph, desc: LayerDesc, weights: torch.Tensor, node_in: torch.Tensor,

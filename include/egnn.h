@@ -44,6 +44,17 @@ typedef enum {
   EGNN_ERR_DEVICE_CHECK = 5   /* a kernel set the status word (see egnn_read_status) */
 } egnn_status;
 
+/* Values of the device status word (egnn_graph::status; first writer wins). */
+enum {
+  EGNN_DEV_BAD_POSITION = 1,      /* a coordinate outside [0, box) or not finite        */
+  EGNN_DEV_SEGMENT_TOO_LARGE = 2, /* an atom with more than 4096 incoming edges         */
+  EGNN_DEV_INDEX_RANGE = 3,       /* a source index outside [0, n_atoms)                */
+  EGNN_DEV_COUNT_MISMATCH = 4,    /* neighbour count and fill passes disagreed           */
+  EGNN_DEV_EDGE_OVERFLOW = 5,     /* more than 2^31 - 1 edges                            */
+  EGNN_DEV_WAIT_TIMEOUT = 6,      /* a bounded wait of a pipelined kernel ran out        */
+  EGNN_DEV_BAD_GRAPH = 7          /* row_ptr not monotone or out of range                */
+};
+
 typedef enum { EGNN_FP32 = 0, EGNN_BF16 = 1 } egnn_dtype;
 
 /* Layer hyper-parameters.  Limits: 0 <= mmax <= min(lmax, 2), lmax <= 6,
@@ -84,11 +95,16 @@ int32_t egnn_wigner_floats(int32_t lmax, int32_t mmax);
 enum { EGNN_WS_BUILD_GRAPH = 0, EGNN_WS_LAYER = 1, EGNN_WS_HAMILTONIAN = 2 };
 
 /* Bytes of device workspace `which` needs (0 allowed).  For EGNN_WS_BUILD_GRAPH
- * only n_atoms matters and desc may be NULL.  For the tensor-core layer and head
- * (bf16, C = 128) the size grows with n_edges by the per-edge message record
- * (4 L C + 4 C sum_{b=1..mmax} (L - b) bytes, 6 KB at lmax 4, mmax 2) plus 4 bytes per
- * edge and head for the attention logits; the gate and A-operand buffers are sized
- * for one range of at most 4096 edge tiles of 128 edges and stop growing beyond it. */
+ * only n_atoms matters and desc may be NULL.  Tensor-core calls (bf16, C = 128), with
+ * L = lmax + 1:
+ *   layer: no per-edge message is stored.  The size grows with n_edges only by two
+ *     partial-softmax records per tile of 128 edges, 2 * 4 (L^2 C + 32) / 128 bytes
+ *     per edge (202 at lmax 4), and with n_atoms by an fp32 accumulator of L^2 C
+ *     values per atom;
+ *   head: grows with n_edges by the per-edge record of the SO(2) outputs
+ *     (4 L C + 4 C sum_{b=1..mmax} (L - b) bytes, 6 KB at lmax 4, mmax 2);
+ * the gate and A-operand buffers of both are sized for one range of at most 4096
+ * edge tiles and stop growing beyond it. */
 size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* desc, int32_t n_atoms,
                             int64_t n_edges);
 
@@ -116,6 +132,18 @@ egnn_status egnn_build_graph(const double* pos, const int32_t* species, int32_t 
                              egnn_graph* g, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /*
+ * egnn_edge_geometry -- recompute every edge's distance and Wigner-D rows of an
+ * existing graph for new positions, keeping its neighbour list (row_ptr, src, shift),
+ * e.g. when atoms moved less than a skin distance since the list was built.
+ *   [MALOQ] Section III-C1 and Fig. 3 (the per-edge rotation to a common axis).
+ * pos  device fp64 [g->n_atoms][3], wrapped into the box as for egnn_build_graph;
+ * box  host fp64 [3].  Degrees stored as g->lmax / g->mmax.  Asynchronous; does not
+ * clear the status word.  A source index outside [0, n_atoms) sets it to
+ * EGNN_DEV_INDEX_RANGE (that edge's rows are left unwritten).
+ */
+egnn_status egnn_edge_geometry(const double* pos, const double box[3], egnn_graph* g, void* cuda_stream);
+
+/*
  * egnn_build_graph_noalloc -- egnn_build_graph without a caller-supplied workspace.
  * The pages have no counterpart to this call; it exists for callers that cannot
  * obtain device memory for a workspace, for example a component that only
@@ -127,8 +155,10 @@ egnn_status egnn_build_graph(const double* pos, const int32_t* species, int32_t 
  * Arguments, outputs and errors are those of egnn_build_graph, plus:
  *   n_atoms above 131072 returns EGNN_ERR_UNSUPPORTED before any work;
  *   the first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any stream
- *   capture.
+ *   device, with that device current) and keeps it for the life of the process;
+ *   make that first call before any stream capture.  The kept address belongs to
+ *   the device's context at that time: after cudaDeviceReset (or any teardown of
+ *   the primary context) do not call this entry point again in the same process.
  * All calls share the one array (whatever stream they use) and the kernels clear
  * what must start at zero, so calls that overlap on the GPU race: order them, for
  * example on one stream.
@@ -158,7 +188,8 @@ egnn_status egnn_build_graph_noalloc(const double* pos, const int32_t* species, 
  *   Input index of x0 is l*2C + c2, of x+-m is (l-m)*2C + c2; output index of y0
  *   is l*C + c, of y+-m is (l-m)*C + c; gate index l*2C + c2.
  * node_in / node_out  device [n_atoms][(lmax+1)^2][C], fp32 or bf16 per dtype;
- *   must not overlap.  An atom without incoming edges gets out = in.
+ *   their byte ranges must be disjoint (any overlap, partial included, returns
+ *   EGNN_ERR_INVALID_ARG).  An atom without incoming edges gets out = in.
  *   weights, node_in and node_out must be 16-byte aligned (EGNN_ERR_INVALID_ARG).
  * g must come from egnn_build_graph with the same lmax/mmax and rcut.
  */
@@ -193,6 +224,15 @@ egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_layer_desc* 
                                     int32_t n_shells, const void* node_emb, float* blocks,
                                     void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* egnn_check_bounded_wait -- diagnostic of the failure path (the pages have no
+ * counterpart).  Every pipelined kernel waits on mbarriers with a time limit and, when
+ * the limit runs out, records EGNN_DEV_WAIT_TIMEOUT in the status word and returns
+ * instead of hanging.  This call runs that same wait routine in a one-thread kernel on
+ * an mbarrier that nothing arrives on, with a limit of `limit_us` microseconds
+ * (1 .. 2,000,000), so the status word of `g` reads EGNN_DEV_WAIT_TIMEOUT afterwards.
+ * Asynchronous on `cuda_stream`; the context stays usable. */
+egnn_status egnn_check_bounded_wait(egnn_graph* g, uint32_t limit_us, void* cuda_stream);
+
 /* Synchronises `cuda_stream`, returns EGNN_ERR_DEVICE_CHECK if the graph's status
  * word is non-zero (its value goes to *code when code != NULL), else EGNN_OK. */
 egnn_status egnn_read_status(const egnn_graph* g, int32_t* code, void* cuda_stream);
@@ -201,10 +241,11 @@ egnn_status egnn_read_status(const egnn_graph* g, int32_t* code, void* cuda_stre
 const char* egnn_status_string(egnn_status s);
 
 /*
- * egnn_profile / egnn_profile_read -- opt-in timing of the SO(2) GEMM kernel of
- * tensor-core egnn_layer_forward calls (a diagnostic; the pages have no counterpart).
+ * egnn_profile / egnn_profile_read -- opt-in timing of the main kernel of tensor-core
+ * egnn_layer_forward calls, the fused SO(2) layer kernel (one launch per range of at
+ * most 4096 edge tiles); a diagnostic, the pages have no counterpart.
  * egnn_profile(1) clears the record and starts recording; egnn_profile(0) stops.
- * While recording, every SO(2) GEMM launch of a layer call is bracketed by two CUDA
+ * While recording, every such launch of a layer call is bracketed by two CUDA
  * events recorded on that call's stream (at most 4096 launches per record; later
  * ones are not recorded).  The events are created on first use, on the device
  * current at the time, and kept until the process exits: use one device per

@@ -100,3 +100,31 @@ def hamiltonian_blocks(pos, box, row_ptr, src, shift, n_emb, W, shells, *, lmax,
     if not blocks:
         return np.zeros((0, n_orb, n_orb))
     return np.concatenate(blocks, axis=0)
+
+
+def assemble_hamiltonian(n_atoms, row_ptr, src, onsite, edge_blocks):
+    """Gamma-point Hamiltonian of the whole structure as a dense matrix (fp64).
+
+    MALOQ Section III-B (Label->Matrix: the predicted blocks placed at their atom
+    pair's rows and columns of H, the orbital template fixing the slices); the
+    review page of arXiv 2507.03840 (one matrix of 104,833 orbitals for the
+    8,064-atom GeSbTe cell).  Readings (the pages give no formula): every atom d
+    owns the rows of its n_orb orbitals; the on-site block of d and the blocks of
+    all its incoming edges s -> d (rows d's orbitals, columns s's) are added at
+    (d, d) and (d, s); periodic images of the same pair sum into one block (the
+    k = 0 matrix).
+
+    onsite[N, n_orb, n_orb]; edge_blocks[E, n_orb, n_orb] in CSR order.
+    Returns H[N n_orb, N n_orb].
+    """
+    onsite = np.asarray(onsite, dtype=np.float64)
+    edge_blocks = np.asarray(edge_blocks, dtype=np.float64)
+    n_orb = onsite.shape[1]
+    H = np.zeros((n_atoms * n_orb, n_atoms * n_orb))
+    for d in range(n_atoms):
+        r = slice(d * n_orb, (d + 1) * n_orb)
+        H[r, r] += onsite[d]
+        for e in range(int(row_ptr[d]), int(row_ptr[d + 1])):
+            s = int(src[e])
+            H[r, s * n_orb:(s + 1) * n_orb] += edge_blocks[e]
+    return H

@@ -11,7 +11,7 @@ Fig. 3); messages are aggregated onto their target nodes (MALOQ Section III);
 the target node owns its incoming edges so attention and aggregation are local
 (review page of arXiv 2507.03840, "What carries the argument").
 
-Readings taken where the pages are silent (every one is listed in the design doc):
+Readings taken where the pages are silent:
   * edge vector r_e = x_s + shift*box - x_d points from the receiver d to the
     sender s; frame R_e with R_e r_e/|r_e| = z-hat (oracle.sh.frame);
   * concatenation order [n_s || n_d] along channels (2C input channels);

@@ -20,6 +20,46 @@ def rel_err(got, ref):
     return float(np.abs(got - ref).max() / (den if den > 0 else 1.0))
 
 
+def check_layer(got, ref, nd, tol, heads=1, bf16_out=None):
+    """Layer output parity, as asserted by every layer test.
+
+    got, ref, nd: [atoms, (lmax+1)^2, C] (GPU output, oracle output, layer input n_d).
+    Normwise-infinity relative error (max|got - ref| / max|ref|) below ``tol``:
+      * on the whole output;
+      * on the update out - n_d, after allowing each element the rounding of a bf16
+        output (2^-8 |ref|, half an ulp), which is relative to |out|, not to the
+        smaller update;
+      * on every block of one degree l and one attention head's channels, for the
+        output and for the update, so that small blocks (high l, one head) are pinned
+        by their own magnitude rather than by the largest block's.
+    Returns the largest of these errors."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    nd = np.asarray(nd, dtype=np.float64)
+    bf16_out = tol > 1e-3 if bf16_out is None else bf16_out
+    diff = np.abs(got - ref)
+    allow = (2.0 ** -8) * np.abs(ref) if bf16_out else np.zeros_like(ref)
+    upd = ref - nd
+
+    def upd_err(sl):
+        den = np.abs(upd[sl]).max()
+        num = max(0.0, float((diff[sl] - allow[sl]).max()))
+        return num / den if den > 0 else num
+
+    errs = {"out": rel_err(got, ref), "update": upd_err(np.s_[:])}
+    L = int(round(np.sqrt(got.shape[1])))
+    C = got.shape[2]
+    hc = C // heads
+    for l in range(L):
+        for h in range(heads):
+            sl = np.s_[:, l * l:(l + 1) * (l + 1), h * hc:(h + 1) * hc]
+            errs[f"out l={l} h={h}"] = rel_err(got[sl], ref[sl])
+            errs[f"update l={l} h={h}"] = upd_err(sl)
+    worst = max(errs, key=errs.get)
+    assert errs[worst] < tol, (worst, errs[worst])
+    return errs[worst]
+
+
 @functools.lru_cache(maxsize=8)
 def cell(name: str, seed: int = 0, n_atoms: int | None = None):
     w = synth.WORKLOADS[name]

@@ -86,14 +86,29 @@ def test_profile_record_starts_empty_and_checks_outputs():
     assert egnn.lib.egnn_profile_read(None, None, None) == egnn.EGNN_ERR_INVALID_ARG
 
 
-def test_layer_workspace_grows_by_the_message_record_per_edge():
-    # tensor-core layer: per edge the y record (y0 fp32, |m| > 0 bf16) and the logits;
-    # the per-range gate and A buffers stop growing once a range is full
+def test_layer_workspace_stores_no_per_edge_message():
+    # fused tensor-core layer: per 128-edge tile two partial-softmax records of
+    # L^2 C + 32 floats; nothing else grows with the edges once a range of tiles is full
     L, C, H = 5, 128, 8
     d = egnn.make_desc(4, 2, C, H, 32, 8.0, "bf16")
-    rec = 4 * L * C + 4 * C * ((L - 1) + (L - 2))
     e1, e2 = 4096 * 128 * 4, 4096 * 128 * 8          # both beyond one full range of tiles
     w1 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 1000, e1)
     w2 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 1000, e2)
+    per_edge = (w2 - w1) / (e2 - e1)
+    assert abs(per_edge - 2 * 4 * (L * L * C + 32) / 128) < 0.01
+    # per atom: one fp32 accumulator of L^2 C values
+    a1 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 10_000, e1)
+    a2 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 20_000, e1)
+    assert abs((a2 - a1) / 10_000 - 4 * L * L * C) < 1.0
+
+
+def test_head_workspace_grows_by_the_message_record_per_edge():
+    # tensor-core head: per edge the y record (y0 fp32, |m| > 0 bf16) and the logits slot
+    L, C, H = 5, 128, 8
+    d = egnn.make_desc(4, 2, C, H, 32, 8.0, "bf16")
+    rec = 4 * L * C + 4 * C * ((L - 1) + (L - 2))
+    e1, e2 = 4096 * 128 * 4, 4096 * 128 * 8
+    w1 = egnn.workspace_bytes(egnn.EGNN_WS_HAMILTONIAN, d, 1000, e1)
+    w2 = egnn.workspace_bytes(egnn.EGNN_WS_HAMILTONIAN, d, 1000, e2)
     per_edge = (w2 - w1) / (e2 - e1)
     assert abs(per_edge - (rec + 4 * H)) < 1.0

@@ -5,7 +5,7 @@ workloads on a seeded sample of destination atoms (the layer is local to each
 destination atom, so a sampled atom's output is exact, not statistical).
 Tolerances: fp32 1e-4, bf16 storage / fp32 accumulation 2e-2, as max relative
 error max|gpu - ref| / max|ref|, applied to the output and to the update
-out - n_d separately."""
+out - n_d, and to each (degree, attention head) block of both (check_layer)."""
 import dataclasses
 
 import numpy as np
@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import synth
-from gpu_helpers import TOL, cell, gpu_graph, oracle_graph, rel_err, sample_atoms, to_dev
+from gpu_helpers import TOL, cell, check_layer, gpu_graph, oracle_graph, rel_err, sample_atoms, to_dev
 from oracle import head as ohead
 from oracle import layer as olayer
 
@@ -47,16 +47,8 @@ def run_layer(egnn, name, w, seed=0, n_atoms=None, atoms=None, bias_std=0.0):
     return got[sel], ref, n[sel]
 
 
-def check(got, ref, nd, tol, bf16_out=None):
-    """Output within tol of max|ref|; the update out - n_d within tol of max|update|
-    after allowing each element the rounding of a bf16 output (half an ulp,
-    2^-8 |ref|), which is relative to |out| rather than to the smaller update."""
-    bf16_out = tol > 1e-3 if bf16_out is None else bf16_out
-    e_out = rel_err(got, ref)
-    allow = (2.0 ** -8) * np.abs(ref) if bf16_out else 0.0
-    e_upd = max(0.0, float((np.abs(got - ref) - allow).max())) / np.abs(ref - nd).max()
-    assert e_out < tol, e_out
-    assert e_upd < tol, e_upd
+def check(got, ref, nd, tol, heads=1):
+    check_layer(got, ref, nd, tol, heads=heads)
 
 
 def test_layer_tiny_fp32_every_atom(egnn):
@@ -76,7 +68,7 @@ def test_layer_small_bf16_every_atom(egnn):
     # 300-atom HfO2-density cell, full C=128, lmax 4: many chunks per atom
     w = synth.WORKLOADS["hfo2_3000"]
     got, ref, nd = run_layer(egnn, "hfo2_3000", w, n_atoms=300, bias_std=0.1)
-    check(got, ref, nd, TOL["bf16"])
+    check(got, ref, nd, TOL["bf16"], heads=w.heads)
 
 
 @pytest.mark.parametrize("name", ["hfo2_3000", "gst_8064", "mixed_12000", "stress_40000"])
@@ -85,7 +77,7 @@ def test_layer_full_size_sampled(egnn, name):
     pos, _, _ = cell(name)
     atoms = np.concatenate([[0, len(pos) - 1], sample_atoms(len(pos), 30, 3)])
     got, ref, nd = run_layer(egnn, name, w, atoms=np.unique(atoms))
-    check(got, ref, nd, TOL["bf16"])
+    check(got, ref, nd, TOL["bf16"], heads=w.heads)
 
 
 def test_layer_isolated_atom_keeps_embedding(egnn):
@@ -119,7 +111,7 @@ def test_layer_bf16_degrees(egnn, lmax, mmax):
     assert g.read_status() == 0
     rp, src, sh = oracle_graph("hfo2_3000", 0, 100)
     ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
-    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"])
+    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"], heads=w.heads)
 
 
 @pytest.mark.parametrize("heads", [1, 16])
@@ -136,7 +128,7 @@ def test_layer_bf16_head_counts(egnn, heads):
     assert g.read_status() == 0
     rp, src, sh = oracle_graph("hfo2_3000", 0, 100)
     ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
-    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"])
+    check(out.float().cpu().numpy().astype(np.float64), ref, n, TOL["bf16"], heads=w.heads)
 
 
 def test_layer_is_deterministic(egnn):
@@ -237,7 +229,7 @@ def test_layer_bf16_fewer_edges_than_one_tile(egnn, n_atoms):
     rp, src, sh = og.neighbour_list_bruteforce(pos, box, w.rcut)
     ref = olayer.layer_forward(pos, box, rp, src, sh, n, W, **_kw(w), heads=w.heads)
     got = out.float().cpu().numpy().astype(np.float64)
-    check(got, ref, n, TOL["bf16"])
+    check(got, ref, n, TOL["bf16"], heads=w.heads)
     np.testing.assert_array_equal(got[-1], n[-1])
 
 

@@ -93,3 +93,47 @@ def test_block_equivariance_under_global_rotation():
         o += 2 * l + 1
     np.testing.assert_allclose(Hb2, Dorb @ Hb @ Dorb.T, atol=1e-10)
     assert np.abs(Hb).max() > 1e-2
+
+
+def test_assembly_two_atoms_by_hand():
+    # two atoms, one s orbital each, edges 1 -> 0 (twice, two images) and 0 -> 1:
+    # H = [[on0, e10a + e10b], [e01, on1]]
+    from oracle.head import assemble_hamiltonian
+    row_ptr = np.array([0, 2, 3])
+    src = np.array([1, 1, 0])
+    onsite = np.array([[[1.5]], [[-2.0]]])
+    edges = np.array([[[0.25]], [[0.5]], [[-0.75]]])
+    H = assemble_hamiltonian(2, row_ptr, src, onsite, edges)
+    np.testing.assert_array_equal(H, [[1.5, 0.75], [-0.75, -2.0]])
+
+
+def test_assembly_symmetric_for_transposed_reverse_edges():
+    # random graph with every edge's reverse carrying the transposed block: H symmetric;
+    # on-site blocks only on the block diagonal; trace from the on-site blocks alone
+    from oracle.head import assemble_hamiltonian
+    rng = np.random.default_rng(4)
+    n, n_orb = 6, 4
+    pairs = [(d, s) for d in range(n) for s in range(n) if d != s and rng.random() < 0.5]
+    pairs = sorted(set(pairs) | {(s, d) for d, s in pairs})
+    blk = {}
+    for d, s in pairs:
+        if (s, d) in blk:
+            blk[(d, s)] = blk[(s, d)].T
+        else:
+            blk[(d, s)] = rng.standard_normal((n_orb, n_orb))
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    src, edges = [], []
+    for d in range(n):
+        for dd, s in pairs:
+            if dd == d:
+                src.append(s)
+                edges.append(blk[(d, s)])
+        row_ptr[d + 1] = len(src)
+    on = rng.standard_normal((n, n_orb, n_orb))
+    on = on + on.transpose(0, 2, 1)
+    H = assemble_hamiltonian(n, row_ptr, np.array(src), on, np.array(edges))
+    np.testing.assert_allclose(H, H.T, atol=0)
+    assert np.isclose(np.trace(H), sum(np.trace(o) for o in on))
+    Hz = assemble_hamiltonian(n, row_ptr, np.array(src), np.zeros_like(on), np.array(edges))
+    for d in range(n):
+        assert np.all(Hz[d * n_orb:(d + 1) * n_orb, d * n_orb:(d + 1) * n_orb] == 0)

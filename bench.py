@@ -407,6 +407,34 @@ def main():
                               "traffic": None if layer_traffic is None else layer_traffic * E,
                               "traffic_note": layer_traffic_note}
 
+    # ---- Label <-> Matrix and Hamiltonian assembly of the step's blocks (timed apart) ----
+    label_rows = None
+    if has_head and rank == 0:
+        def timed(fn, reps=5):
+            fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+        onsite = torch.zeros(len(pos_np), w.n_orb, w.n_orb, dtype=torch.float32, device=dev)
+        all_blocks = torch.cat([onsite, blocks])      # on-site and edge blocks of the cell
+        labels = egnn.blocks_to_labels(all_blocks, w.shells)
+        t_m2l = timed(lambda: egnn.blocks_to_labels(all_blocks, w.shells))
+        t_l2m = timed(lambda: egnn.labels_to_blocks(labels, w.shells))
+        t_asm = timed(lambda: egnn.assemble_hamiltonian(g, onsite, blocks))
+        nb = all_blocks.shape[0]
+        label_rows = {
+            "template_orbitals": w.n_orb, "blocks": nb, "labels_per_block": egnn.label_count(w.shells),
+            "matrix_to_label_ms": t_m2l, "matrix_to_label_atoms_per_s": len(pos_np) / (t_m2l / 1e3),
+            "label_to_matrix_ms": t_l2m, "h_assembly_ms": t_asm,
+            "h_orbitals": len(pos_np) * w.n_orb,
+            "bytes_per_conversion": nb * (w.n_orb * w.n_orb + egnn.label_count(w.shells)) * 4,
+            "note": "one structure's on-site + edge blocks per conversion; the pages quote 7.3e5-1.2e6 "
+                    "atoms/s Matrix->Label on one GH200 (context, other hardware)"}
+
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
@@ -460,7 +488,7 @@ def main():
                        "step": "build_graph + layers + hamiltonian head",
                        "l2": "inputs larger than L2 (per step >1 GB of Wigner rows and blocks)",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "label_matrix": label_rows,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libegnn.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "graph.cu", "so2_simt.cu", "so2_tc.cu", "so2_fused.cu"]
+SOURCES = ["api.cu", "graph.cu", "so2_simt.cu", "so2_tc.cu", "so2_fused.cu", "labels.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -223,7 +223,7 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_at
 // partial records per edge tile.  Nothing in it is stored per edge except the
 // records (2 (L^2 C + 32) floats per 128 edges).
 struct LayerWorkspace {
-  size_t wprep, gate, x, stash, acc, slots, total;
+  size_t wprep, gate, x, stash, edst, acc, slots, total;
   int rec_floats;
 };
 
@@ -241,7 +241,8 @@ LayerWorkspace layer_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_
   w.gate = align_up((size_t)P.wprep_bytes, 1024);
   w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
   w.stash = w.x + align_up(tch * P.nch * 16384, 1024);
-  w.acc = w.stash + align_up((size_t)kTcMaxGrid * L * 128 * C * 2, 1024);
+  w.edst = w.stash + align_up((size_t)kTcMaxGrid * L * 128 * C * 2, 1024);
+  w.acc = w.edst + align_up(E * 4, 1024);
   w.slots = w.acc + align_up(N * L * L * C * 4, 1024);
   w.total = w.slots + align_up(n_tiles * 2 * (size_t)w.rec_floats * 4, 1024) + 1024;
   return w;
@@ -292,6 +293,7 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
     T.gates = (__nv_bfloat16*)(ws + lw.gate);
     T.X = ws + lw.x;
     T.stash = (__nv_bfloat16*)(ws + lw.stash);
+    T.edge_dst = (int32_t*)(ws + lw.edst);
     T.acc_g = (float*)(ws + lw.acc);
     T.slots = (float*)(ws + lw.slots);
     T.rec_floats = lw.rec_floats;
@@ -333,12 +335,16 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
 
 uint8_t* align1024(void* p) { return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023); }
 
+}  // namespace
+
 // ---------------- Clebsch-Gordan tables (library side) ----------------
 // Complex coefficients <j1 m1 j2 m2 | J M> by Racah's closed formula, then the
 // unitary change to the real basis of egnn.h (real_m = sum_mu U[m][mu] Y^mu,
 // Y^mu with the Condon-Shortley phase):  C_real = (U_la (x) U_lb) C U_L^dagger.
 // The result is real up to one global phase, removed before the sign rule
 // (first non-zero entry of column M = -L positive).
+namespace {
+
 double fact(int n) {
   double r = 1;
   for (int i = 2; i <= n; ++i) r *= i;
@@ -378,6 +384,9 @@ std::complex<double> real_from_complex(int m, int mu) {
   return 0.0;
 }
 
+}  // namespace
+
+// Real Clebsch-Gordan matrix C^L(la, lb), row-major [(2la+1)(2lb+1)][2L+1], appended to out.
 void real_cg(int la, int lb, int L, std::vector<float>& out) {
   int na = 2 * la + 1, nb = 2 * lb + 1, nl = 2 * L + 1;
   std::vector<std::complex<double>> C(na * nb * nl);
@@ -414,7 +423,6 @@ void real_cg(int la, int lb, int L, std::vector<float>& out) {
   for (double x : R) out.push_back((float)x);
 }
 
-}  // namespace
 
 extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* desc, int32_t n_atoms,
                                        int64_t n_edges) {
@@ -426,6 +434,10 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
         return layer_workspace(desc, n_edges, n_atoms).total;
       return 256;
+    case EGNN_WS_LABELS:
+      return 64 * 1024;
+    case EGNN_WS_ASSEMBLY:
+      return (size_t)(n_atoms > 0 ? n_atoms : 0) * 4 + 256;
     case EGNN_WS_HAMILTONIAN:
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
         return tc_workspace(desc, n_edges, n_atoms).total + 64 * 1024;

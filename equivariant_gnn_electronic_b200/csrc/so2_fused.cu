@@ -72,10 +72,18 @@ struct EpiSmem {
 __device__ __forceinline__ void epi_bar() { tc::bar_sync(kEpiBar, 256); }
 __device__ __forceinline__ void group_bar(int g) { tc::bar_sync(2 + g, 128); }
 
-__device__ __forceinline__ float* seg_target(const TcParams& P, const EpiSmem* es, int t, int k) {
+// What the epilogue helpers need of the launch parameters, passed by value (registers)
+// rather than as a reference to the kernel's parameter block.
+struct EpiArgs {
+  float* slots;
+  float* acc_g;
+  int C, L2, rec_floats;
+};
+
+__device__ __forceinline__ float* seg_target(const EpiArgs& A, const EpiSmem* es, int t, int k) {
   const int slot = es->seg_slot[k];
-  return slot >= 0 ? P.slots + ((size_t)t * 2 + slot) * P.rec_floats
-                   : P.acc_g + (size_t)es->seg_d[k] * P.L2 * P.C;
+  return slot >= 0 ? A.slots + ((size_t)t * 2 + slot) * A.rec_floats
+                   : A.acc_g + (size_t)es->seg_d[k] * A.L2 * A.C;
 }
 
 __device__ __forceinline__ int pad4(int x) { return (x + 3) & ~3; }
@@ -112,13 +120,13 @@ __device__ __forceinline__ void flush(float* tg, int C, float2* acc) {
 // segment's record).  The thread's stash row holds its channel's 128 edges
 // contiguously (bf16), read 32 edges at a time with the next 32 in flight.
 template <int NL>
-__device__ __noinline__ void y0_degree(const TcParams& P, const EpiSmem* es, int t, int l, int c, int hh,
+__device__ __noinline__ void y0_degree(const EpiArgs A, const EpiSmem* es, int t, int l, int c, int hh,
                                        int nvalid, int DZ, int offz, const uint4* st_row) {
   float2 acc[(NL + 1) / 2];
 #pragma unroll
   for (int i = 0; i < (NL + 1) / 2; ++i) acc[i] = make_float2(0.f, 0.f);
   int k = 0, nb = es->seg_b[1];
-  const int C = P.C;
+  const int C = A.C;
   const size_t roff = (size_t)(l * l) * C + c;
   uint4 cur[4], nxt[4];
 #pragma unroll
@@ -145,7 +153,7 @@ __device__ __noinline__ void y0_degree(const TcParams& P, const EpiSmem* es, int
           const int e = j8 + i;
           if (e >= nvalid) break;
           if (e == nb) {
-            flush<NL, false>(seg_target(P, es, t, k) + roff, C, acc);
+            flush<NL, false>(seg_target(A, es, t, k) + roff, C, acc);
             ++k;
             nb = es->seg_b[k + 1];
           }
@@ -156,14 +164,14 @@ __device__ __noinline__ void y0_degree(const TcParams& P, const EpiSmem* es, int
 #pragma unroll
     for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
   }
-  flush<NL, false>(seg_target(P, es, t, k) + roff, C, acc);
+  flush<NL, false>(seg_target(A, es, t, k) + roff, C, acc);
 }
 
 // 8 edges of a (+b, -b) pass: acc[m'] += p_e (D^l_e[+b, m'] y+_e + D^l_e[-b, m'] y-_e).
 // The Wigner rows of the pass are dw[e][2][NP] (shared memory).
 template <int NL>
 __device__ __forceinline__ void pm_edges(const EpiSmem* es, const float* dw, int hh, int j, int nvalid,
-                                         const uint32_t* y, float2* acc, int& k, int& nb, const TcParams& P,
+                                         const uint32_t* y, float2* acc, int& k, int& nb, const EpiArgs& A,
                                          int t, size_t roff) {
   constexpr int NP = (NL + 3) & ~3;
   if (j + 8 <= nb && j + 8 <= nvalid) {
@@ -181,7 +189,7 @@ __device__ __forceinline__ void pm_edges(const EpiSmem* es, const float* dw, int
     const int e = j + i;
     if (e >= nvalid) break;
     if (e == nb) {
-      flush<NL, true>(seg_target(P, es, t, k) + roff, P.C, acc);
+      flush<NL, true>(seg_target(A, es, t, k) + roff, A.C, acc);
       ++k;
       nb = es->seg_b[k + 1];
     }
@@ -196,13 +204,13 @@ __device__ __forceinline__ void pm_edges(const EpiSmem* es, const float* dw, int
 // tb + 256), read 8 edges at a time with the next 8 in flight; sums added into each
 // destination segment's record.
 template <int NL>
-__device__ __noinline__ void pm_degree(const TcParams& P, const EpiSmem* es, const float* dw, int t, int l, int c,
+__device__ __noinline__ void pm_degree(const EpiArgs A, const EpiSmem* es, const float* dw, int t, int l, int c,
                                        int hh, int nvalid, uint32_t tb) {
   float2 acc[(NL + 1) / 2];
 #pragma unroll
   for (int i = 0; i < (NL + 1) / 2; ++i) acc[i] = make_float2(0.f, 0.f);
   int k = 0, nb = es->seg_b[1];
-  const size_t roff = (size_t)(l * l) * P.C + c;
+  const size_t roff = (size_t)(l * l) * A.C + c;
   uint32_t ya[16], yb[16];   // [0, 8) y+, [8, 16) y- of 8 edges
   tc::tmem_ld8_issue(tb, ya);
   tc::tmem_ld8_issue(tb + 128, ya + 8);
@@ -214,18 +222,18 @@ __device__ __noinline__ void pm_degree(const TcParams& P, const EpiSmem* es, con
       tc::tmem_ld8_issue(tb + j + 8, yb);
       tc::tmem_ld8_issue(tb + 128 + j + 8, yb + 8);
     }
-    pm_edges<NL>(es, dw, hh, j, nvalid, ya, acc, k, nb, P, t, roff);
+    pm_edges<NL>(es, dw, hh, j, nvalid, ya, acc, k, nb, A, t, roff);
     if (!more1) break;
     tc::tmem_ld_wait8x2(yb, yb + 8);
     if (more2) {
       tc::tmem_ld8_issue(tb + j + 16, ya);
       tc::tmem_ld8_issue(tb + 128 + j + 16, ya + 8);
     }
-    pm_edges<NL>(es, dw, hh, j + 8, nvalid, yb, acc, k, nb, P, t, roff);
+    pm_edges<NL>(es, dw, hh, j + 8, nvalid, yb, acc, k, nb, A, t, roff);
     if (!more2) break;
     tc::tmem_ld_wait8x2(ya, ya + 8);
   }
-  flush<NL, true>(seg_target(P, es, t, k) + roff, P.C, acc);
+  flush<NL, true>(seg_target(A, es, t, k) + roff, A.C, acc);
 }
 
 __device__ __forceinline__ bool own_deg(const TcParams& P, int g, int l) { return ((P.own_b >> l) & 1) == g; }
@@ -277,9 +285,8 @@ __device__ __noinline__ void m0_stash(uint32_t tb, __nv_bfloat16* row) {
 // Lp[q][e][h] += sum_c A[h][l C + c] SiLU(y0_e[l, c]), by warp-level mma.sync on
 // 16-edge x 16-channel blocks of SiLU(y0) staged in the warp's tile T (bf16, 16-byte
 // pieces of a row swizzled by ((row >> 1) & 3)); each lane owns fixed (e, h) entries.
-__device__ __noinline__ void m0_logits(const TcParams& P, uint32_t tb, int l, int q, int lane, float* Lp,
-                                       uint16_t* T, uint32_t T_u32) {
-  const int C = P.C, H = P.H, L = P.L;
+__device__ __noinline__ void m0_logits(const __nv_bfloat16* Amat, int C, int H, int L, uint32_t tb, int l, int q,
+                                       int lane, float* Lp, uint16_t* T, uint32_t T_u32) {
   const int nnt = H > 8 ? 2 : 1;
   uint32_t bf[2][2][2];
 #pragma unroll
@@ -289,7 +296,7 @@ __device__ __noinline__ void m0_logits(const TcParams& P, uint32_t tb, int l, in
       const int n = nt * 8 + (lane >> 2);
       const int k0 = l * C + q * 32 + kt * 16 + 2 * (lane & 3);
       const bool ok = n < H && nt < nnt;
-      const uint32_t* ap = reinterpret_cast<const uint32_t*>(P.A + (size_t)n * L * C + k0);
+      const uint32_t* ap = reinterpret_cast<const uint32_t*>(Amat + (size_t)n * L * C + k0);
       bf[kt][nt][0] = ok ? __ldg(ap) : 0u;
       bf[kt][nt][1] = ok ? __ldg(ap + 4) : 0u;
     }
@@ -494,6 +501,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     __nv_bfloat16* stash = P.stash + (size_t)blockIdx.x * L * 128 * C;
     float* dg = es->dbuf + g * kDGroup;                    // this group's Wigner rows
+    const EpiArgs EA{P.slots, P.acc_g, P.C, P.L2, P.rec_floats};
     int DZ = 0;
     for (int l = 0; l < L; ++l) DZ += pad4(2 * l + 1);
     uint32_t ip = 0;
@@ -502,19 +510,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       const long long e0 = (long long)t * 128;
       const int nvalid = (int)(E - e0 < 128 ? E - e0 : 128);
       // ---- destination segments of the tile (group 0 threads: one per edge) ----
-      if (et < 128) {
-        int d = -1;
-        if (et < nvalid) {
-          const long long e = e0 + et;
-          int lo = 0, hi = P.n_atoms;
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
-          }
-          d = lo;
-        }
-        es->dst[et] = d;
-      }
+      if (et < 128) es->dst[et] = et < nvalid ? P.edge_dst[e0 + et] : -1;
       epi_bar();
       {
         const bool start = et < nvalid && (et == 0 || es->dst[et] != es->dst[et - 1]);
@@ -565,7 +561,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           const int l = ps.n_off / 128 + rb;
           const uint32_t tb = tl + buf * 256 + rb * 128;
           if (g == 1) m0_stash(tb, stash + ((size_t)l * C + c) * 128);
-          else m0_logits(P, tb, l, q, lane, Lp, T, T_u32);
+          else m0_logits(P.A, C, H, L, tb, l, q, lane, Lp, T, T_u32);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
@@ -575,10 +571,8 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       epi_bar();
       if (et < 128) {
         for (int h = 0; h < H; ++h) {
-          float a = __bfloat162float(P.bA[h]);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) a += Lp[(w * 128 + et) * H + h];
-          es->pw[et * 16 + h] = a;
+          float a = Lp[et * H + h] + Lp[(128 + et) * H + h] + Lp[(256 + et) * H + h] + Lp[(384 + et) * H + h];
+          es->pw[et * 16 + h] = a + __bfloat162float(P.bA[h]);
         }
       }
       epi_bar();
@@ -603,14 +597,15 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       // ---- rows m = 0 of every D^l for the tile (one edge per thread of group 0) ----
       if (et < nvalid && et < 128) {
         const float* wr = P.wig + (size_t)(e0 + et) * P.wfl;
-        float* dz = es->dbuf + et * DZ;
+        const uint32_t dz = tc::smem_u32(es->dbuf + et * DZ);
         int off = 0;
         for (int l = 0; l < L; ++l) {
           const int ml = l < P.mmax ? l : P.mmax, dl = 2 * l + 1;
           const float* row = wr + P.woff[l] + ml * dl;   // row m = 0 of D^l
-          for (int m = 0; m < dl; ++m) dz[off + m] = __ldg(row + m);
+          for (int m = 0; m < dl; ++m) tc::cp_async4(dz + 4 * (off + m), row + m);
           off += pad4(dl);
         }
+        tc::cp_async_wait_all();
       }
       epi_bar();
       // ---- y0 from the stash, degrees of this group: first contribution of each record ----
@@ -620,13 +615,13 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           if (own_deg(P, g, l)) {
             const uint4* st_row = reinterpret_cast<const uint4*>(stash + ((size_t)l * C + c) * 128);
             switch (l) {
-              case 0: y0_degree<1>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 1: y0_degree<3>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 2: y0_degree<5>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 3: y0_degree<7>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 4: y0_degree<9>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 5: y0_degree<11>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              default: y0_degree<13>(P, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 0: y0_degree<1>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 1: y0_degree<3>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 2: y0_degree<5>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 3: y0_degree<7>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 4: y0_degree<9>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 5: y0_degree<11>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              default: y0_degree<13>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
             }
           }
           offz += pad4(2 * l + 1);
@@ -661,12 +656,12 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           tc::tc_fence_after();
           const uint32_t tb = tl + buf * 256;
           switch (l) {
-            case 1: pm_degree<3>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 2: pm_degree<5>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 3: pm_degree<7>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 4: pm_degree<9>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 5: pm_degree<11>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
-            default: pm_degree<13>(P, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 1: pm_degree<3>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 2: pm_degree<5>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 3: pm_degree<7>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 4: pm_degree<9>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 5: pm_degree<11>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            default: pm_degree<13>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
           }
           tc::tc_fence_before();
           tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
@@ -765,6 +760,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Tc
           __float2bfloat16_rn(__bfloat162float(P.node_in[o + (size_t)i * C]) + acc[i] * inv);
 }
 
+// Destination atom of every edge (one warp per atom; consecutive edges, coalesced stores).
+__global__ void edge_dst_kernel(const int32_t* __restrict__ row_ptr, int n_atoms, int32_t* __restrict__ dst) {
+  const int d = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (d >= n_atoms) return;
+  for (int e = row_ptr[d] + lane; e < row_ptr[d + 1]; e += 32) dst[e] = d;
+}
+
 size_t fused_smem_total() {
   return kXS * kXBytes + kWS * kWBytes + ((sizeof(EpiSmem) + 15) & ~(size_t)15) + sizeof(FusedCtl) + 1024;
 }
@@ -781,9 +783,10 @@ cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*)
 
 size_t layer_fused_smem_bytes(int, int) { return fused_smem_total(); }
 
-// Weight prep, then per range of edge tiles: gate GEMM -> rotate -> fused SO(2) layer;
-// then the destinations that cross tile boundaries or have no edges.
+// Destination of every edge, weight prep, then per range of edge tiles: gates and rotation
+// -> fused SO(2) layer; then the destinations that cross tile boundaries or have none.
 cudaError_t launch_layer_fused(const TcParams& P, const TcWeights& W, cudaStream_t st) {
+  if (P.n_edges > 0) edge_dst_kernel<<<(P.n_atoms * 32 + 255) / 256, 256, 0, st>>>(P.row_ptr, P.n_atoms, P.edge_dst);
   cudaError_t err = launch_tc_pipeline(P, W, st, fused_consumer, nullptr, true);
   if (err != cudaSuccess) return err;
   combine_kernel<<<P.n_atoms, 128, 0, st>>>(P);

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 struct So2Params {
   int n_atoms;
   long long n_edges;
@@ -46,3 +48,7 @@ size_t so2_simt_smem_bytes(const So2Params& P, int te);
 int so2_simt_pick_te(const So2Params& P, int head_labels);
 cudaError_t launch_layer_simt(So2Params P, So2Weights W, cudaStream_t st);
 cudaError_t launch_head_simt(So2Params P, So2Weights W, HeadTables T, cudaStream_t st);
+
+// Real Clebsch-Gordan matrix C^L(la, lb) of the basis of egnn.h, row-major
+// [(2la+1)(2lb+1)][2L+1], appended to `out` (api.cu).
+void real_cg(int la, int lb, int L, std::vector<float>& out);

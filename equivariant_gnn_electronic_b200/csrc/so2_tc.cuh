@@ -68,6 +68,7 @@ struct TcParams {
   // being the unnormalised weighted sum [L^2][C], then the per-head softmax maximum [16]
   // and denominator [16] of the tile's part of the segment.
   __nv_bfloat16* stash;
+  int32_t* edge_dst;             // destination atom of every edge (fused layer)
   float* acc_g;
   float* slots;
   int rec_floats;

@@ -18,12 +18,13 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libegnn.so
 EGNN_OK, EGNN_ERR_INVALID_ARG, EGNN_ERR_CAPACITY, EGNN_ERR_UNSUPPORTED, EGNN_ERR_CUDA, \
     EGNN_ERR_DEVICE_CHECK = range(6)
 EGNN_FP32, EGNN_BF16 = 0, 1
-EGNN_WS_BUILD_GRAPH, EGNN_WS_LAYER, EGNN_WS_HAMILTONIAN = 0, 1, 2
+EGNN_WS_BUILD_GRAPH, EGNN_WS_LAYER, EGNN_WS_HAMILTONIAN, EGNN_WS_LABELS, EGNN_WS_ASSEMBLY = 0, 1, 2, 3, 4
 
 EXPORTED = (
     "egnn_wigner_floats", "egnn_workspace_bytes", "egnn_build_graph", "egnn_layer_forward",
     "egnn_hamiltonian_blocks", "egnn_read_status", "egnn_status_string", "egnn_build_graph_noalloc",
     "egnn_profile", "egnn_profile_read", "egnn_edge_geometry", "egnn_check_bounded_wait",
+    "egnn_label_count", "egnn_blocks_to_labels", "egnn_labels_to_blocks", "egnn_assemble_hamiltonian",
 )
 EGNN_DEV_BAD_POSITION, EGNN_DEV_SEGMENT_TOO_LARGE, EGNN_DEV_INDEX_RANGE, EGNN_DEV_COUNT_MISMATCH, \
     EGNN_DEV_EDGE_OVERFLOW, EGNN_DEV_WAIT_TIMEOUT, EGNN_DEV_BAD_GRAPH = range(1, 8)
@@ -77,6 +78,13 @@ def _load():
     lib.egnn_edge_geometry.restype = i32
     lib.egnn_check_bounded_wait.argtypes = [ctypes.POINTER(GraphStruct), ctypes.c_uint32, vp]
     lib.egnn_check_bounded_wait.restype = i32
+    lib.egnn_label_count.argtypes = [ctypes.POINTER(i32), i32]
+    lib.egnn_label_count.restype = i32
+    for name in ("egnn_blocks_to_labels", "egnn_labels_to_blocks"):
+        getattr(lib, name).argtypes = [vp, i64, ctypes.POINTER(i32), i32, vp, vp, sz, vp]
+        getattr(lib, name).restype = i32
+    lib.egnn_assemble_hamiltonian.argtypes = [ctypes.POINTER(GraphStruct), vp, vp, i32, vp, vp, vp, i64, vp, sz, vp]
+    lib.egnn_assemble_hamiltonian.restype = i32
     lib.egnn_profile.argtypes = [i32]
     lib.egnn_profile.restype = i32
     lib.egnn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), ctypes.POINTER(i64)]
@@ -232,6 +240,50 @@ def check_bounded_wait(graph: Graph, limit_us: int, stream=None) -> None:
     """Run the pipelined kernels' bounded wait on an mbarrier nothing arrives on."""
     _check(lib.egnn_check_bounded_wait(ctypes.byref(graph.s), int(limit_us), _stream(stream)),
            "egnn_check_bounded_wait")
+
+
+def label_count(shells: Sequence[int]) -> int:
+    sh = (ctypes.c_int32 * len(shells))(*shells)
+    return int(lib.egnn_label_count(sh, len(shells)))
+
+
+def _template_call(name, x: torch.Tensor, n: int, shells: Sequence[int], out: torch.Tensor, stream):
+    ws = torch.empty(workspace_bytes(EGNN_WS_LABELS, None, 0, 0), dtype=torch.uint8, device=x.device)
+    sh = (ctypes.c_int32 * len(shells))(*shells)
+    _check(getattr(lib, name)(_ptr(x), n, sh, len(shells), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), name)
+    return out
+
+
+def blocks_to_labels(blocks: torch.Tensor, shells: Sequence[int], stream=None) -> torch.Tensor:
+    """Matrix -> Label: [n, n_orb, n_orb] fp32 -> [n, n_lab] fp32."""
+    assert blocks.dtype == torch.float32 and blocks.is_contiguous()
+    out = torch.empty(blocks.shape[0], label_count(shells), dtype=torch.float32, device=blocks.device)
+    return _template_call("egnn_blocks_to_labels", blocks, blocks.shape[0], shells, out, stream)
+
+
+def labels_to_blocks(labels: torch.Tensor, shells: Sequence[int], stream=None) -> torch.Tensor:
+    """Label -> Matrix: [n, n_lab] fp32 -> [n, n_orb, n_orb] fp32."""
+    assert labels.dtype == torch.float32 and labels.is_contiguous()
+    n_orb = sum(2 * l + 1 for l in shells)
+    out = torch.empty(labels.shape[0], n_orb, n_orb, dtype=torch.float32, device=labels.device)
+    return _template_call("egnn_labels_to_blocks", labels, labels.shape[0], shells, out, stream)
+
+
+def assemble_hamiltonian(graph: Graph, onsite: torch.Tensor, edge_blocks: torch.Tensor, stream=None):
+    """k = 0 Hamiltonian as block-sparse rows: (bsr_row_ptr [N+1], bsr_col [nnzb],
+    bsr_val [nnzb, n_orb, n_orb]) with the arrays sized for N + E blocks (trim by
+    bsr_row_ptr[N])."""
+    n, n_orb = graph.n_atoms, onsite.shape[1]
+    cap = n + graph.n_edges
+    dev = onsite.device
+    row_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(cap, dtype=torch.int32, device=dev)
+    val = torch.empty(cap, n_orb, n_orb, dtype=torch.float32, device=dev)
+    ws = torch.empty(workspace_bytes(EGNN_WS_ASSEMBLY, None, n, 0), dtype=torch.uint8, device=dev)
+    _check(lib.egnn_assemble_hamiltonian(ctypes.byref(graph.s), _ptr(onsite), _ptr(edge_blocks), n_orb,
+                                         _ptr(row_ptr), _ptr(col), _ptr(val), cap, _ptr(ws), ws.numel(),
+                                         _stream(stream)), "egnn_assemble_hamiltonian")
+    return row_ptr, col, val
 
 
 def layer_forward(graph: Graph, desc: LayerDesc, weights: torch.Tensor, node_in: torch.Tensor,

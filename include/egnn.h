@@ -92,15 +92,21 @@ typedef struct {
 int32_t egnn_wigner_floats(int32_t lmax, int32_t mmax);
 
 /* Which call a workspace is for. */
-enum { EGNN_WS_BUILD_GRAPH = 0, EGNN_WS_LAYER = 1, EGNN_WS_HAMILTONIAN = 2 };
+enum {
+  EGNN_WS_BUILD_GRAPH = 0,
+  EGNN_WS_LAYER = 1,
+  EGNN_WS_HAMILTONIAN = 2,
+  EGNN_WS_LABELS = 3,       /* egnn_labels_to_blocks / egnn_blocks_to_labels (64 KB)  */
+  EGNN_WS_ASSEMBLY = 4      /* egnn_assemble_hamiltonian (4 bytes per atom)          */
+};
 
 /* Bytes of device workspace `which` needs (0 allowed).  For EGNN_WS_BUILD_GRAPH
  * only n_atoms matters and desc may be NULL.  Tensor-core calls (bf16, C = 128), with
  * L = lmax + 1:
  *   layer: no per-edge message is stored.  The size grows with n_edges only by two
- *     partial-softmax records per tile of 128 edges, 2 * 4 (L^2 C + 32) / 128 bytes
- *     per edge (202 at lmax 4), and with n_atoms by an fp32 accumulator of L^2 C
- *     values per atom;
+ *     partial-softmax records per tile of 128 edges and a 4-byte destination index
+ *     per edge, 2 * 4 (L^2 C + 32) / 128 + 4 bytes per edge (206 at lmax 4), and
+ *     with n_atoms by an fp32 accumulator of L^2 C values per atom;
  *   head: grows with n_edges by the per-edge record of the SO(2) outputs
  *     (4 L C + 4 C sum_{b=1..mmax} (L - b) bytes, 6 KB at lmax 4, mmax 2);
  * the gate and A-operand buffers of both are sized for one range of at most 4096
@@ -232,6 +238,49 @@ egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_layer_desc* 
  * (1 .. 2,000,000), so the status word of `g` reads EGNN_DEV_WAIT_TIMEOUT afterwards.
  * Asynchronous on `cuda_stream`; the context stays usable. */
 egnn_status egnn_check_bounded_wait(egnn_graph* g, uint32_t limit_us, void* cuda_stream);
+
+/*
+ * Label <-> block conversion ([MALOQ] Section III-B1, Eq. (1); Section III-B2 and
+ * Fig. 2(b-d): Matrix -> Label for training targets, Label -> Matrix for the
+ * prediction, on the GPU, driven by the orbital template).
+ * Orbital template: shell_l host int32 [n_shells] (1..16 shells, each l <= 3, at most
+ * 32 orbitals), shared by both atoms of a block.  Labels per block: for L = 0 .. 2 max l,
+ * M = -L..L, then k over the shell pairs (a, b) with |l_a - l_b| <= L <= l_a + l_b
+ * (lexicographic, a outer): the layout egnn_hamiltonian_blocks uses.  Label
+ * h[L, M, k] = sum_{i, j} C^L_{(l_a i)(l_b j), M} H[(a, i), (b, j)] with the real
+ * Clebsch-Gordan matrices of egnn_hamiltonian_blocks; since each C^L has orthonormal
+ * columns and together they are square per pair, the two calls are inverse.
+ * blocks device fp32 [n][n_orb][n_orb]; labels device fp32 [n][egnn_label_count(...)].
+ * workspace: egnn_workspace_bytes(EGNN_WS_LABELS, ...) bytes of device memory (tables).
+ * Asynchronous on `cuda_stream`.  Errors: bad template EGNN_ERR_UNSUPPORTED, null
+ * pointers or small workspace EGNN_ERR_INVALID_ARG.
+ */
+int32_t egnn_label_count(const int32_t* shell_l, int32_t n_shells);
+egnn_status egnn_blocks_to_labels(const float* blocks, int64_t n, const int32_t* shell_l, int32_t n_shells,
+                                  float* labels, void* workspace, size_t ws_bytes, void* cuda_stream);
+egnn_status egnn_labels_to_blocks(const float* labels, int64_t n, const int32_t* shell_l, int32_t n_shells,
+                                  float* blocks, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * egnn_assemble_hamiltonian -- the k = 0 Hamiltonian of the structure as block-sparse
+ * rows (BSR) from on-site and per-edge orbital blocks ([MALOQ] Section III-B2, the
+ * Label -> Matrix reconstruction of the whole matrix; [DEGNN] one matrix of 104,833
+ * orbitals for the 8,064-atom cell).
+ * Row block d (orbitals of atom d) holds the on-site block onsite[d] at column d and,
+ * for every distinct source atom s of d's incoming edges, the sum of those edges'
+ * blocks at column s (periodic images of one pair add up; images of d itself add to
+ * the on-site block).  Column blocks ascend within a row; sums run in edge order, so
+ * the result is deterministic.
+ * onsite device fp32 [n_atoms][n_orb][n_orb]; edge_blocks device fp32
+ * [n_edges][n_orb][n_orb] in the graph's edge order (e.g. from egnn_hamiltonian_blocks).
+ * bsr_row_ptr device int32 [n_atoms + 1]; bsr_col device int32 [capacity]; bsr_val device
+ * fp32 [capacity][n_orb][n_orb].  capacity >= n_atoms + n_edges is required (else
+ * EGNN_ERR_CAPACITY) and always suffices; the block count is bsr_row_ptr[n_atoms].
+ * workspace: egnn_workspace_bytes(EGNN_WS_ASSEMBLY, NULL, n_atoms, 0) bytes.  Asynchronous.
+ */
+egnn_status egnn_assemble_hamiltonian(const egnn_graph* g, const float* onsite, const float* edge_blocks,
+                                      int32_t n_orb, int32_t* bsr_row_ptr, int32_t* bsr_col, float* bsr_val,
+                                      int64_t capacity, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /* Synchronises `cuda_stream`, returns EGNN_ERR_DEVICE_CHECK if the graph's status
  * word is non-zero (its value goes to *code when code != NULL), else EGNN_OK. */

@@ -88,14 +88,15 @@ def test_profile_record_starts_empty_and_checks_outputs():
 
 def test_layer_workspace_stores_no_per_edge_message():
     # fused tensor-core layer: per 128-edge tile two partial-softmax records of
-    # L^2 C + 32 floats; nothing else grows with the edges once a range of tiles is full
+    # L^2 C + 32 floats, and a 4-byte destination index per edge; nothing else grows
+    # with the edges once a range of tiles is full
     L, C, H = 5, 128, 8
     d = egnn.make_desc(4, 2, C, H, 32, 8.0, "bf16")
     e1, e2 = 4096 * 128 * 4, 4096 * 128 * 8          # both beyond one full range of tiles
     w1 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 1000, e1)
     w2 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 1000, e2)
     per_edge = (w2 - w1) / (e2 - e1)
-    assert abs(per_edge - 2 * 4 * (L * L * C + 32) / 128) < 0.01
+    assert abs(per_edge - (2 * 4 * (L * L * C + 32) / 128 + 4)) < 0.01
     # per atom: one fp32 accumulator of L^2 C values
     a1 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 10_000, e1)
     a2 = egnn.workspace_bytes(egnn.EGNN_WS_LAYER, d, 20_000, e1)

@@ -330,12 +330,12 @@ def main():
         return x
 
     # Our kernels per step (tensor-core path): graph build 7 (cell_assign, scan, cell_fill,
-    # nbr_count, scan, nbr_fill, wigner); per layer prep_weights, then gate + rotate +
-    # layer_fused per range of edge tiles, then combine; the head prep_weights, gate +
-    # rotate + so2_gemm per range, head_label.
+    # nbr_count, scan, nbr_fill, wigner); per layer edge_dst and prep_weights, then
+    # gate_rotate + layer_fused per range of edge tiles, then combine; the head
+    # prep_weights, gate_rotate + so2_gemm per range, head_label.
     n_tiles = (E + 127) // 128
     n_ranges = max(1, -(-n_tiles // 4096))
-    launches_per_step = 7 + w.n_layers * (2 + 3 * n_ranges) + ((2 + 3 * n_ranges) if has_head else 0)
+    launches_per_step = 7 + w.n_layers * (3 + 2 * n_ranges) + ((2 + 2 * n_ranges) if has_head else 0)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -399,7 +399,8 @@ def main():
                 "timing": "CUDA events recorded by the library around each launch, on its stream, "
                           "inside the timed region",
                 "messages_in_hbm": False}
-    roofline["layer_call"] = {"kernels": "prep_weights, (gate, rotate, layer_fused) per edge-tile range, combine",
+    roofline["layer_call"] = {"kernels": "edge_dst, prep_weights, (gate_rotate, layer_fused) per edge-tile "
+                                         "range, combine",
                               "ms": 1e3 * layer_avg_s, "tflops": layer_tf, "frac": layer_tf / peak,
                               "frac_of_burst": layer_tf / peak_burst,
                               "flops_per_call": layer_flops, "flops_counted": "radial MLP + SO(2), 8.528 MFLOP/edge",

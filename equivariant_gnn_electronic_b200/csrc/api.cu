@@ -197,7 +197,7 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
 }
 
 struct TcWorkspace {
-  size_t wprep, gate, x, y, logits, af, total;
+  size_t wprep, x, y, total;
 };
 
 TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_atoms) {
@@ -208,22 +208,19 @@ TcWorkspace tc_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_t n_at
   size_t E = n_edges > 0 ? (size_t)n_edges : 0;
   const size_t tch = (size_t)tc_chunk_tiles((int)((E + 127) / 128));
   w.wprep = 0;
-  w.gate = align_up((size_t)P.wprep_bytes, 1024);
-  w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
+  w.x = align_up((size_t)P.wprep_bytes, 1024);
   w.y = w.x + align_up(tch * P.nch * 16384, 1024);
-  w.logits = w.y + align_up(E * (size_t)P.y_row_bytes, 1024);
   (void)n_atoms;
-  w.af = w.logits + align_up(E * d->heads * 4, 1024);
-  w.total = w.af + align_up((size_t)d->heads * (d->lmax + 1) * d->channels * 4, 1024) + 1024;
+  w.total = w.y + align_up(E * (size_t)P.y_row_bytes, 1024) + 1024;
   return w;
 }
 
-// Workspace of the fused tensor-core layer: prepared weights, the gates and A tiles of
-// one range of edge tiles, the per-CTA y0 stash, per-atom accumulators and two
+// Workspace of the fused tensor-core layer: prepared weights, the A tiles of one range
+// of edge tiles, the per-CTA y0 stash, per-atom accumulators and two
 // partial records per edge tile.  Nothing in it is stored per edge except the
 // records (2 (L^2 C + 32) floats per 128 edges).
 struct LayerWorkspace {
-  size_t wprep, gate, x, stash, edst, acc, slots, total;
+  size_t wprep, x, stash, edst, acc, slots, total;
   int rec_floats;
 };
 
@@ -238,8 +235,7 @@ LayerWorkspace layer_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_
   const size_t tch = (size_t)tc_chunk_tiles((int)n_tiles);
   w.rec_floats = (int)(L * L * C + 32);
   w.wprep = 0;
-  w.gate = align_up((size_t)P.wprep_bytes, 1024);
-  w.x = w.gate + align_up(tch * 128 * P.gcols * 2, 1024);
+  w.x = align_up((size_t)P.wprep_bytes, 1024);
   w.stash = w.x + align_up(tch * P.nch * 16384, 1024);
   w.edst = w.stash + align_up((size_t)kTcMaxGrid * L * 128 * C * 2, 1024);
   w.acc = w.edst + align_up(E * 4, 1024);
@@ -252,7 +248,7 @@ LayerWorkspace layer_workspace(const egnn_layer_desc* d, int64_t n_edges, int32_
 // workspace (label mode with `mult`; the fused layer's layout with `layer`); returns
 // false if the pass plan does not fit.
 bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_desc* desc, const So2Weights& W,
-             const void* node_in, void* node_out, uint8_t* ws, int with_logits, const int* mult = nullptr,
+             const void* node_in, void* node_out, uint8_t* ws, const int* mult = nullptr,
              bool layer = false) {
   TcWorkspace wl = tc_workspace(desc, g->n_edges, g->n_atoms);
   memset(&T, 0, sizeof(T));
@@ -278,7 +274,6 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   T.dist = g->dist;
   T.wig = g->wigner;
   T.status = g->status;
-  T.with_logits = with_logits;
   T.node_in = (const __nv_bfloat16*)node_in;
   T.node_out = (__nv_bfloat16*)node_out;
   for (int l = 0; l <= desc->lmax; ++l) T.woff[l] = egnn_wig_off(l, desc->mmax);
@@ -290,7 +285,6 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
   if (layer) {
     const LayerWorkspace lw = layer_workspace(desc, g->n_edges, g->n_atoms);
     T.wprep = ws + lw.wprep;
-    T.gates = (__nv_bfloat16*)(ws + lw.gate);
     T.X = ws + lw.x;
     T.stash = (__nv_bfloat16*)(ws + lw.stash);
     T.edge_dst = (int32_t*)(ws + lw.edst);
@@ -320,11 +314,8 @@ bool fill_tc(TcParams& T, TcWeights& TW, const egnn_graph* g, const egnn_layer_d
     }
   } else {
     T.wprep = ws + wl.wprep;
-    T.gates = (__nv_bfloat16*)(ws + wl.gate);
     T.X = ws + wl.x;
     T.Y = ws + wl.y;
-    T.logits = (float*)(ws + wl.logits);
-    T.Af = (float*)(ws + wl.af);
   }
   TW.W2 = (const __nv_bfloat16*)W.W2;
   TW.W0 = (const __nv_bfloat16*)W.W0;
@@ -435,12 +426,12 @@ extern "C" size_t egnn_workspace_bytes(int32_t which, const egnn_layer_desc* des
         return layer_workspace(desc, n_edges, n_atoms).total;
       return 256;
     case EGNN_WS_LABELS:
-      return 64 * 1024;
+      return 1024 * 1024;
     case EGNN_WS_ASSEMBLY:
       return (size_t)(n_atoms > 0 ? n_atoms : 0) * 4 + 256;
     case EGNN_WS_HAMILTONIAN:
       if (desc && check_desc(desc) == EGNN_OK && tc_eligible(desc))
-        return tc_workspace(desc, n_edges, n_atoms).total + 64 * 1024;
+        return tc_workspace(desc, n_edges, n_atoms).total + 1024 * 1024;
       return 64 * 1024;
     default:
       return 0;
@@ -473,7 +464,7 @@ extern "C" egnn_status egnn_layer_forward(const egnn_graph* g, const egnn_layer_
     carve_so2(W, (const char*)weights, desc, true);
     TcParams T;
     TcWeights TW;
-    fill_tc(T, TW, g, desc, W, node_in, node_out, ws, 1, nullptr, true);
+    fill_tc(T, TW, g, desc, W, node_in, node_out, ws, nullptr, true);
     EGNN_CUDA_TRY(launch_layer_fused(T, TW, st));
     return EGNN_OK;
   }
@@ -574,13 +565,77 @@ extern "C" egnn_status egnn_hamiltonian_blocks(const egnn_graph* g, const egnn_l
     memset(&probe, 0, sizeof(probe));
     const bool label = tc_plan(desc, probe, mult) && probe.y_row_bytes <= y_bytes;
     TcWeights TW;
-    if (!fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, 0, label ? mult : nullptr))
+    if (!fill_tc(TP, TW, g, desc, W, node_emb, nullptr, ws_tc, label ? mult : nullptr))
       return EGNN_ERR_UNSUPPORTED;
     for (int Lc = 0; Lc < 8; ++Lc) TP.U[Lc] = (const __nv_bfloat16*)W.U[Lc];
     HeadUPtrs Up;
     for (int Lc = 0; Lc < 8; ++Lc) Up.U[Lc] = (const __nv_bfloat16*)W.U[Lc];
     if (head_tc_smem_bytes(TP, T.n_lab, 1) > 200 * 1024) return EGNN_ERR_UNSUPPORTED;
-    EGNN_CUDA_TRY(launch_head_tc(TP, TW, T, Up, blocks, st));
+    HeadLabelTabs LT;
+    memset(&LT, 0, sizeof(LT));
+    if (label) {
+      // label q: its rotate-back terms (Wigner offset, record offset); block entry q: its
+      // (label, Clebsch-Gordan coefficient) terms
+      const int norb = T.n_orb, nb = norb * norb, R = kTcPairRows;
+      std::vector<int> lab((size_t)T.n_lab * 11, 0), tptr(nb + 1, 0);
+      std::vector<int2> terms;
+      int lb[3][8];
+      for (int b = 0; b < 3; ++b) {
+        int acc = 0;
+        for (int l = 0; l < 8; ++l) {
+          lb[b][l] = acc;
+          if (l >= b && l <= desc->lmax) acc += mult[l];
+        }
+      }
+      for (int q0 = 0; q0 < T.n_lab; ++q0) {
+        int q = q0, Lq = 0;
+        while (q >= (2 * Lq + 1) * mult[Lq]) q -= (2 * Lq + 1) * mult[Lq++];
+        const int M = q / mult[Lq], k = q - M * mult[Lq];
+        const int ml = Lq < desc->mmax ? Lq : desc->mmax, dl = 2 * Lq + 1, D = TP.woff[Lq] + M;
+        int* o = &lab[(size_t)q0 * 11];
+        o[0] = 2 * ml + 1;
+        o[1] = D + ml * dl;
+        o[6] = TP.hroff[0] + lb[0][Lq] + k;
+        int j = 1;
+        for (int b = 1; b <= ml; ++b) {
+          const int r = lb[b][Lq] + k, qq = r / R, w = r - qq * R, rest = TP.hnr[b] - R * qq;
+          const int npq = rest >= R ? R : ((rest + 15) & ~15), base = TP.hroff[b] + 2 * R * qq + w;
+          o[1 + j] = D + (ml + b) * dl;
+          o[6 + j++] = base;
+          o[1 + j] = D + (ml - b) * dl;
+          o[6 + j++] = base + npq;
+        }
+      }
+      for (int q = 0; q < nb; ++q) {
+        const int ri = q / norb, cj = q - ri * norb, a = T.orb_shell[ri], b = T.orb_shell[cj];
+        const int la = T.shell_l[a], lbb = T.shell_l[b], ia = ri - T.shell_off[a], jb = cj - T.shell_off[b];
+        for (int Lc = abs(la - lbb); Lc <= la + lbb; ++Lc) {
+          const int k = kidx[(a * n_shells + b) * 8 + Lc];
+          const float* cgm = cg.data() + T.cg_off[(la * 4 + lbb) * 8 + Lc] + (ia * (2 * lbb + 1) + jb) * (2 * Lc + 1);
+          for (int M = 0; M < 2 * Lc + 1; ++M) {
+            int2 tm;
+            tm.x = T.lab_off[Lc] + M * mult[Lc] + k;
+            memcpy(&tm.y, &cgm[M], 4);
+            terms.push_back(tm);
+          }
+        }
+        tptr[q + 1] = (int)terms.size();
+      }
+      const size_t o_lab = (off + cg.size() * sizeof(float) + 15) & ~(size_t)15;
+      const size_t o_ptr = (o_lab + lab.size() * 4 + 15) & ~(size_t)15;
+      const size_t o_term = (o_ptr + tptr.size() * 4 + 15) & ~(size_t)15;
+      if ((size_t)(wsp - (char*)workspace) + o_term + terms.size() * 8 > ws_bytes) return EGNN_ERR_INVALID_ARG;
+      EGNN_CUDA_TRY(cudaMemcpyAsync(wsp + o_lab, lab.data(), lab.size() * 4, cudaMemcpyHostToDevice, st));
+      EGNN_CUDA_TRY(cudaMemcpyAsync(wsp + o_ptr, tptr.data(), tptr.size() * 4, cudaMemcpyHostToDevice, st));
+      EGNN_CUDA_TRY(cudaMemcpyAsync(wsp + o_term, terms.data(), terms.size() * 8, cudaMemcpyHostToDevice, st));
+      LT.n_lab = T.n_lab;
+      LT.n_orb = norb;
+      LT.n_term = (int)terms.size();
+      LT.lab = (const int*)(wsp + o_lab);
+      LT.term_ptr = (const int*)(wsp + o_ptr);
+      LT.term = (const int2*)(wsp + o_term);
+    }
+    EGNN_CUDA_TRY(launch_head_tc(TP, TW, T, Up, LT, blocks, st));
     return EGNN_OK;
   }
   So2Params P;

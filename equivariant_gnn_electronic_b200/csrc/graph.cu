@@ -323,6 +323,150 @@ __global__ void __launch_bounds__(128) wigner_kernel(
   }
 }
 
+// ---- Wigner rows for lmax <= 4: the recursion unrolled per degree (registers), the
+// rows of a CTA's 128 edges staged in shared memory and written out contiguously ----
+__host__ __device__ constexpr int wig_floats_c(int lmax, int mmax) {
+  int o = 0;
+  for (int k = 0; k <= lmax; ++k) o += (2 * (k < mmax ? k : mmax) + 1) * (2 * k + 1);
+  return o;
+}
+
+// Ivanic-Ruedenberg P function of degree l from the previous degree's matrix.
+template <int l>
+__device__ __forceinline__ float ir_P(const float (&D1)[3][3], const float* prev, int i, int a, int b) {
+  constexpr int dp = 2 * l - 1;
+  const float r1 = D1[i + 1][2], rm1 = D1[i + 1][0], r0 = D1[i + 1][1];
+  if (b == l) return r1 * prev[(a + l - 1) * dp + (2 * l - 2)] - rm1 * prev[(a + l - 1) * dp];
+  if (b == -l) return r1 * prev[(a + l - 1) * dp] + rm1 * prev[(a + l - 1) * dp + (2 * l - 2)];
+  return r0 * prev[(a + l - 1) * dp + (b + l - 1)];
+}
+
+// D^l (row-major (2l+1)^2) from D^{l-1} and D^1, every index a compile-time constant.
+template <int l>
+__device__ __forceinline__ void ir_level(const float (&D1)[3][3], const float* prev, float* cur) {
+  constexpr int dc = 2 * l + 1;
+#pragma unroll
+  for (int m = -l; m <= l; ++m) {
+    const int am = m < 0 ? -m : m;
+    const float dm0 = (m == 0) ? 1.f : 0.f;
+#pragma unroll
+    for (int nn = -l; nn <= l; ++nn) {
+      const float den = (nn > -l && nn < l) ? (float)((l + nn) * (l - nn)) : (float)(2 * l * (2 * l - 1));
+      const float u = sqrtf((float)((l + m) * (l - m)) / den);
+      const float v = 0.5f * sqrtf((1.f + dm0) * (float)((l + am - 1) * (l + am)) / den) * (1.f - 2.f * dm0);
+      const float wv = (float)((l - am - 1) * (l - am));
+      const float w = (m == 0 || wv <= 0.f) ? 0.f : -0.5f * sqrtf(wv / den);
+      float val = 0.f;
+      if (l + m != 0 && l - m != 0) val += u * ir_P<l>(D1, prev, 0, m, nn);
+      if (v != 0.f) {
+        float V;
+        if (m == 0) V = ir_P<l>(D1, prev, 1, 1, nn) + ir_P<l>(D1, prev, -1, -1, nn);
+        else if (m > 0)
+          V = ir_P<l>(D1, prev, 1, m - 1, nn) * (m == 1 ? 1.41421356237f : 1.f) -
+              (m == 1 ? 0.f : ir_P<l>(D1, prev, -1, -m + 1, nn));
+        else
+          V = (m == -1 ? 0.f : ir_P<l>(D1, prev, 1, m + 1, nn)) +
+              ir_P<l>(D1, prev, -1, -m - 1, nn) * (m == -1 ? 1.41421356237f : 1.f);
+        val += v * V;
+      }
+      if (m != 0 && l - am - 1 > 0) {
+        const float W = m > 0 ? ir_P<l>(D1, prev, 1, m + 1, nn) + ir_P<l>(D1, prev, -1, -m - 1, nn)
+                              : ir_P<l>(D1, prev, 1, m - 1, nn) - ir_P<l>(D1, prev, -1, -m + 1, nn);
+        val += w * W;
+      }
+      cur[(m + l) * dc + (nn + l)] = val;
+    }
+  }
+}
+
+// Kept rows |m| <= min(l, MM) of D^l into the edge's staged record.
+template <int l, int MM>
+__device__ __forceinline__ void keep_rows(const float* Dl, float* row) {
+  constexpr int ml = l < MM ? l : MM, dc = 2 * l + 1, o = wig_floats_c(l - 1, MM);
+#pragma unroll
+  for (int m = -ml; m <= ml; ++m)
+#pragma unroll
+    for (int j = 0; j < dc; ++j) row[o + (m + ml) * dc + j] = Dl[(m + l) * dc + j];
+}
+
+// Edges per CTA of the tile kernel: 128 when their staged rows fit 48 KB, else 64.
+template <int LM, int MM>
+constexpr int wig_tile_edges() { return 128 * wig_floats_c(LM, MM) * 4 <= 48 * 1024 ? 128 : 64; }
+
+template <int LM, int MM>
+__global__ void __launch_bounds__(128) wigner_tile_kernel(
+    const double* __restrict__ pos, int n, const int32_t* __restrict__ row_ptr,
+    const int32_t* __restrict__ src, const int8_t* __restrict__ shift, long long n_edges, double bx,
+    double by, double bz, float* __restrict__ dist, float* __restrict__ wig, int32_t* status) {
+  constexpr int WFL = wig_floats_c(LM, MM), TE = wig_tile_edges<LM, MM>();
+  __shared__ float rows[TE * WFL];
+  __shared__ int ok[TE];
+  const long long e0 = (long long)blockIdx.x * TE, e = e0 + threadIdx.x;
+  const int nvalid = (int)(n_edges - e0 < TE ? n_edges - e0 : TE);
+  float* row = rows + threadIdx.x * WFL;
+  if (threadIdx.x < TE) ok[threadIdx.x] = 0;
+  if (threadIdx.x < TE && e < n_edges) {
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (row_ptr[mid] <= e) lo = mid; else hi = mid;
+    }
+    const int d = lo, s = src[e];
+    if (s < 0 || s >= n) {
+      egnn_flag(status, EGNN_DEV_INDEX_RANGE);
+    } else {
+      ok[threadIdx.x] = 1;
+      const double rx = __dsub_rn(__dadd_rn(pos[3 * s + 0], __dmul_rn((double)shift[3 * e + 0], bx)), pos[3 * d + 0]);
+      const double ry = __dsub_rn(__dadd_rn(pos[3 * s + 1], __dmul_rn((double)shift[3 * e + 1], by)), pos[3 * d + 1]);
+      const double rz = __dsub_rn(__dadd_rn(pos[3 * s + 2], __dmul_rn((double)shift[3 * e + 2], bz)), pos[3 * d + 2]);
+      const double r = sqrt(rx * rx + ry * ry + rz * rz);
+      dist[e] = (float)r;
+      const double x = rx / r, y = ry / r, z = rz / r;
+      const double rho = sqrt(x * x + y * y);
+      double ca = 1.0, sa = 0.0;
+      if (rho > 0.0) {
+        ca = x / rho;
+        sa = y / rho;
+      }
+      // R = R_y(-beta) R_z(-alpha); D^1 in the (y, z, x) component order
+      const double cb = z, sb = rho;
+      const double R[3][3] = {{cb * ca, cb * sa, -sb}, {-sa, ca, 0.0}, {sb * ca, sb * sa, cb}};
+      const int p[3] = {1, 2, 0};
+      float D1[3][3];
+#pragma unroll
+      for (int i = 0; i < 3; ++i)
+#pragma unroll
+        for (int j = 0; j < 3; ++j) D1[i][j] = (float)R[p[i]][p[j]];
+      row[0] = 1.0f;
+      if constexpr (LM >= 1) {
+        const float* D1f = &D1[0][0];
+        keep_rows<1, MM>(D1f, row);
+        if constexpr (LM >= 2) {
+          float D2[25];
+          ir_level<2>(D1, D1f, D2);
+          keep_rows<2, MM>(D2, row);
+          if constexpr (LM >= 3) {
+            float D3[49];
+            ir_level<3>(D1, D2, D3);
+            keep_rows<3, MM>(D3, row);
+            if constexpr (LM >= 4) {
+              float D4[81];
+              ir_level<4>(D1, D3, D4);
+              keep_rows<4, MM>(D4, row);
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // the CTA's edges are contiguous in the output: coalesced copy (edges with a bad
+  // source index are left unwritten, as in the per-thread path)
+  float* out = wig + e0 * WFL;
+  for (int i = threadIdx.x; i < nvalid * WFL; i += blockDim.x)
+    if (ok[i / WFL]) out[i] = rows[i];
+}
+
 }  // namespace
 
 extern "C" int32_t egnn_wigner_floats(int32_t lmax, int32_t mmax) {
@@ -336,6 +480,31 @@ size_t egnn_graph_workspace_bytes(int32_t n_atoms) {
   size_t ints = n /*atom_cell*/ + (ncell + 1) /*cell_count*/ + (ncell + 1) /*cell_start*/ +
                 ncell /*cell_fill*/ + n /*cell_atoms*/ + n /*counts*/ + 64;
   return ints * sizeof(int32_t) + 256;
+}
+
+// Wigner rows of every edge: the unrolled tile kernel up to lmax 4, the per-thread
+// recursion beyond.
+static cudaError_t launch_wigner(const double* pos, int n_atoms, const egnn_graph* g, long long E,
+                                 const double box[3], int lmax, int mmax, cudaStream_t st) {
+  const int blocks = (int)((E + 127) / 128);
+  switch (mmax * 8 + lmax) {
+#define EGNN_WT_CASE(LMv, MMv)                                                                         \
+  case MMv * 8 + LMv:                                                                                 \
+    wigner_tile_kernel<LMv, MMv><<<(int)((E + wig_tile_edges<LMv, MMv>() - 1) / wig_tile_edges<LMv, MMv>()), \
+                                   wig_tile_edges<LMv, MMv>(), 0, st>>>(pos, n_atoms, g->row_ptr, g->src, g->shift, E, \
+                                                         box[0], box[1], box[2], g->dist, g->wigner,  \
+                                                         g->status);                                  \
+    return cudaGetLastError();
+    EGNN_WT_CASE(0, 0) EGNN_WT_CASE(1, 0) EGNN_WT_CASE(2, 0) EGNN_WT_CASE(3, 0) EGNN_WT_CASE(4, 0)
+    EGNN_WT_CASE(1, 1) EGNN_WT_CASE(2, 1) EGNN_WT_CASE(3, 1) EGNN_WT_CASE(4, 1)
+    EGNN_WT_CASE(2, 2) EGNN_WT_CASE(3, 2) EGNN_WT_CASE(4, 2)
+#undef EGNN_WT_CASE
+    default:
+      break;
+  }
+  wigner_kernel<<<blocks, 128, 0, st>>>(pos, n_atoms, g->row_ptr, g->src, g->shift, E, box[0], box[1], box[2], lmax,
+                                        mmax, egnn_wigner_floats(lmax, mmax), g->dist, g->wigner, g->status);
+  return cudaGetLastError();
 }
 
 extern "C" egnn_status egnn_build_graph(const double* pos, const int32_t* species, int32_t n_atoms,
@@ -411,11 +580,7 @@ extern "C" egnn_status egnn_build_graph(const double* pos, const int32_t* specie
   if (E == 0) return EGNN_OK;
   nbr_fill_kernel<<<n_atoms, kFillThreads, 0, st>>>(pos, n_atoms, G, atom_cell, cell_start, cell_atoms,
                                                     g->row_ptr, g->src, g->shift, g->capacity, g->status);
-  int wfl = egnn_wigner_floats(lmax, mmax);
-  wigner_kernel<<<(int)((E + 127) / 128), 128, 0, st>>>(pos, n_atoms, g->row_ptr, g->src, g->shift, E,
-                                                         box[0], box[1], box[2], lmax, mmax, wfl,
-                                                         g->dist, g->wigner, g->status);
-  EGNN_CUDA_TRY(cudaGetLastError());
+  EGNN_CUDA_TRY(launch_wigner(pos, n_atoms, g, E, box, lmax, mmax, st));
   return EGNN_OK;
 }
 
@@ -430,12 +595,7 @@ extern "C" egnn_status egnn_edge_geometry(const double* pos, const double box[3]
     if (!(box[k] > 0.0) || !(box[k] < 1e12)) return EGNN_ERR_INVALID_ARG;
   if (g->n_edges == 0) return EGNN_OK;
   cudaStream_t st = (cudaStream_t)cuda_stream;
-  const long long E = g->n_edges;
-  wigner_kernel<<<(int)((E + 127) / 128), 128, 0, st>>>(pos, g->n_atoms, g->row_ptr, g->src, g->shift, E, box[0],
-                                                         box[1], box[2], g->lmax, g->mmax,
-                                                         egnn_wigner_floats(g->lmax, g->mmax), g->dist, g->wigner,
-                                                         g->status);
-  EGNN_CUDA_TRY(cudaGetLastError());
+  EGNN_CUDA_TRY(launch_wigner(pos, g->n_atoms, g, g->n_edges, box, g->lmax, g->mmax, st));
   return EGNN_OK;
 }
 

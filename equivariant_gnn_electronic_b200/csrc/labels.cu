@@ -12,10 +12,10 @@
 // for the 8,064-atom GeSbTe cell.
 //
 // Kernels:
-//   labels_to_blocks  CTA per group of blocks; labels staged in shared memory; one
-//                     thread per matrix element sums its pair's labels through C^L.
-//   blocks_to_labels  CTA per group of blocks; blocks staged in shared memory; one
-//                     thread per label sums its pair's block through C^L.
+//   apply_terms       both directions: a group of blocks (or label vectors) staged in
+//                     shared memory, one thread per output element (matrix element, or
+//                     label) summing its precomputed Clebsch-Gordan terms; the term
+//                     lists are built on the host from the orbital template.
 //   h_count / h_scan / h_fill  block-sparse rows of the k = 0 Hamiltonian: row block d
 //                     holds the on-site block of d and, per distinct source atom s of
 //                     d's incoming edges, the sum of those edges' blocks (periodic
@@ -30,136 +30,155 @@
 
 namespace {
 
-constexpr int kLabLmax = 6;   // labels up to L = 2 * 3 (shells up to f)
 
 struct LabelTables {
   int n_shells, n_orb, n_lab, lmax;
-  int mult[8], lab_off[8];
-  int shell_l[16], shell_off[17], orb_shell[32];
-  int cg_off[4 * 4 * 8];
-  const int* kidx;     // [(a * n_shells + b) * 8 + L] -> k
-  const int* pair;     // [lab_off-free index: L * 256 + k] -> a * 16 + b
-  const float* cg;
+  int n_term;             // Clebsch-Gordan terms of one block (both directions have as many)
+  const int* b_ptr;       // [n_orb^2 + 1] terms of each block entry ...
+  const int2* b_term;     // ... (label index, coefficient as float bits)
+  const int* l_ptr;       // [n_lab + 1] terms of each label ...
+  const int2* l_term;     // ... (block entry index, coefficient as float bits)
 };
 
-// Builds the template tables on the host; the device arrays go to `ws` (asynchronous
+// Builds the template's term lists on the host and copies them into `ws` (asynchronous
 // copies on `st` from pageable host memory, staged before the call returns).
 egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T, void* ws, size_t ws_bytes,
                         cudaStream_t st) {
   if (!shell_l || n_shells < 1 || n_shells > 16) return EGNN_ERR_INVALID_ARG;
   memset(&T, 0, sizeof(T));
   T.n_shells = n_shells;
-  int o = 0, lmax = 0;
+  int o = 0, lmax = 0, shell_off[17];
   for (int a = 0; a < n_shells; ++a) {
     const int l = shell_l[a];
     if (l < 0 || l > 3) return EGNN_ERR_UNSUPPORTED;
     if (o + 2 * l + 1 > 32) return EGNN_ERR_UNSUPPORTED;
-    T.shell_l[a] = l;
-    T.shell_off[a] = o;
-    for (int i = 0; i < 2 * l + 1; ++i) T.orb_shell[o + i] = a;
+    shell_off[a] = o;
     o += 2 * l + 1;
     lmax = 2 * l > lmax ? 2 * l : lmax;
   }
-  T.shell_off[n_shells] = o;
   T.n_orb = o;
   T.lmax = lmax;
-  std::vector<int> kidx(n_shells * n_shells * 8, 0), pair(8 * 256, 0);
+  // label order: L, then M, then k over the pairs (a, b) containing L (a outer)
+  int mult[8] = {0}, lab_off[8] = {0};
+  std::vector<int> kidx(n_shells * n_shells * 8, 0);
   for (int a = 0; a < n_shells; ++a)
     for (int b = 0; b < n_shells; ++b)
-      for (int L = abs(shell_l[a] - shell_l[b]); L <= shell_l[a] + shell_l[b]; ++L) {
-        pair[L * 256 + T.mult[L]] = a * 16 + b;
-        kidx[(a * n_shells + b) * 8 + L] = T.mult[L]++;
-      }
+      for (int L = abs(shell_l[a] - shell_l[b]); L <= shell_l[a] + shell_l[b]; ++L)
+        kidx[(a * n_shells + b) * 8 + L] = mult[L]++;
   int lab = 0;
-  for (int L = 0; L < 8; ++L) {
-    T.lab_off[L] = lab;
-    if (L <= lmax) lab += (2 * L + 1) * T.mult[L];
+  for (int L = 0; L <= lmax; ++L) {
+    lab_off[L] = lab;
+    lab += (2 * L + 1) * mult[L];
   }
   T.n_lab = lab;
-  std::vector<float> cg;
-  for (int la = 0; la <= 3; ++la)
-    for (int lb = 0; lb <= 3; ++lb)
+  const int norb = o, nb = norb * norb;
+  // (label, entry, coefficient) of every Clebsch-Gordan term of a block
+  std::vector<int> t_lab, t_ent;
+  std::vector<float> t_cg;
+  for (int a = 0; a < n_shells; ++a)
+    for (int b = 0; b < n_shells; ++b) {
+      const int la = shell_l[a], lb = shell_l[b];
       for (int L = abs(la - lb); L <= la + lb; ++L) {
-        T.cg_off[(la * 4 + lb) * 8 + L] = (int)cg.size();
+        std::vector<float> cg;
         real_cg(la, lb, L, cg);
+        const int k = kidx[(a * n_shells + b) * 8 + L];
+        for (int ia = 0; ia < 2 * la + 1; ++ia)
+          for (int jb = 0; jb < 2 * lb + 1; ++jb)
+            for (int M = 0; M < 2 * L + 1; ++M) {
+              t_lab.push_back(lab_off[L] + M * mult[L] + k);
+              t_ent.push_back((shell_off[a] + ia) * norb + shell_off[b] + jb);
+              t_cg.push_back(cg[(ia * (2 * lb + 1) + jb) * (2 * L + 1) + M]);
+            }
       }
-  const size_t b0 = kidx.size() * 4, b1 = (b0 + 15) & ~(size_t)15;
-  const size_t b2 = b1 + pair.size() * 4, b3 = (b2 + 15) & ~(size_t)15;
-  if (!ws || ws_bytes < b3 + cg.size() * 4) return EGNN_ERR_INVALID_ARG;
+    }
+  const int nt = (int)t_cg.size();
+  T.n_term = nt;
+  // CSR by entry and by label (stable order: the sums run in a fixed order)
+  std::vector<int> bptr(nb + 1, 0), lptr(lab + 1, 0);
+  for (int i = 0; i < nt; ++i) {
+    ++bptr[t_ent[i] + 1];
+    ++lptr[t_lab[i] + 1];
+  }
+  for (int i = 0; i < nb; ++i) bptr[i + 1] += bptr[i];
+  for (int i = 0; i < lab; ++i) lptr[i + 1] += lptr[i];
+  std::vector<int2> bterm(nt), lterm(nt);
+  std::vector<int> bfill(bptr.begin(), bptr.end() - 1), lfill(lptr.begin(), lptr.end() - 1);
+  for (int i = 0; i < nt; ++i) {
+    int2 x;
+    memcpy(&x.y, &t_cg[i], 4);
+    x.x = t_lab[i];
+    bterm[bfill[t_ent[i]]++] = x;
+    x.x = t_ent[i];
+    lterm[lfill[t_lab[i]]++] = x;
+  }
+  const size_t o1 = ((nb + 1) * 4 + 15) & ~(size_t)15, o2 = o1 + (size_t)nt * 8;
+  const size_t o3 = o2 + (((lab + 1) * 4 + 15) & ~(size_t)15), need = o3 + (size_t)nt * 8;
+  if (!ws || ws_bytes < need) return EGNN_ERR_INVALID_ARG;
   char* w = (char*)ws;
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w, kidx.data(), b0, cudaMemcpyHostToDevice, st));
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w + b1, pair.data(), pair.size() * 4, cudaMemcpyHostToDevice, st));
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w + b3, cg.data(), cg.size() * 4, cudaMemcpyHostToDevice, st));
-  T.kidx = (const int*)w;
-  T.pair = (const int*)(w + b1);
-  T.cg = (const float*)(w + b3);
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w, bptr.data(), (nb + 1) * 4, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o1, bterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o2, lptr.data(), (lab + 1) * 4, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o3, lterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
+  T.b_ptr = (const int*)w;
+  T.b_term = (const int2*)(w + o1);
+  T.l_ptr = (const int*)(w + o2);
+  T.l_term = (const int2*)(w + o3);
   return EGNN_OK;
 }
 
-// Label -> block: one thread per matrix element of `te` blocks staged per CTA.
-__global__ void __launch_bounds__(256) labels_to_blocks_kernel(const float* __restrict__ labels, long long n,
-                                                               const __grid_constant__ LabelTables T, int te,
-                                                               float* __restrict__ blocks) {
-  extern __shared__ float lsm[];   // [te][n_lab]
-  const int nlab = T.n_lab, norb = T.n_orb, nb = norb * norb;
+// out[item][q] = sum over the terms of q of coefficient * in[item][index], for `te` items
+// per group staged in shared memory (persistent CTAs; the term list staged once per CTA
+// when it fits).  One thread per output element q, looping over the group's items.
+__global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restrict__ in, int nin, long long n,
+                                                          const int* __restrict__ ptr, const int2* __restrict__ term,
+                                                          int nout, int nterm, int staged, int te,
+                                                          float* __restrict__ out) {
+  extern __shared__ float tsm[];
+  int* s_ptr = reinterpret_cast<int*>(tsm);
+  int2* s_term = reinterpret_cast<int2*>(s_ptr + (staged ? ((nout + 2) & ~1) : 0));
+  float* In = reinterpret_cast<float*>(s_term + (staged ? nterm : 0));   // [te][nin]
+  const int tid = threadIdx.x, nt = blockDim.x;
+  if (staged) {
+    for (int i = tid; i <= nout; i += nt) s_ptr[i] = ptr[i];
+    for (int i = tid; i < nterm; i += nt) s_term[i] = term[i];
+  } else {
+    s_ptr = const_cast<int*>(ptr);
+    s_term = const_cast<int2*>(term);
+  }
   for (long long g0 = (long long)blockIdx.x * te; g0 < n; g0 += (long long)gridDim.x * te) {
     const int ne = (int)min((long long)te, n - g0);
     __syncthreads();
-    for (int i = threadIdx.x; i < ne * nlab; i += blockDim.x) lsm[i] = labels[g0 * nlab + i];
+    for (int i = tid; i < ne * nin; i += nt) In[i] = in[g0 * nin + i];
     __syncthreads();
-    for (int i = threadIdx.x; i < ne * nb; i += blockDim.x) {
-      const int e = i / nb, q = i - e * nb;
-      const int ri = q / norb, cj = q - ri * norb;
-      const int a = T.orb_shell[ri], b = T.orb_shell[cj];
-      const int la = T.shell_l[a], lb = T.shell_l[b];
-      const int ia = ri - T.shell_off[a], jb = cj - T.shell_off[b];
-      float v = 0.f;
-      for (int L = abs(la - lb); L <= la + lb; ++L) {
-        const int k = T.kidx[(a * T.n_shells + b) * 8 + L], mult = T.mult[L];
-        const float* c = T.cg + T.cg_off[(la * 4 + lb) * 8 + L] + (ia * (2 * lb + 1) + jb) * (2 * L + 1);
-        const float* h = lsm + e * nlab + T.lab_off[L] + k;
-        for (int M = 0; M < 2 * L + 1; ++M) v = fmaf(c[M], h[M * mult], v);
+    for (int q = tid; q < nout; q += nt) {
+      const int t0 = s_ptr[q], t1 = s_ptr[q + 1];
+      for (int e = 0; e < ne; ++e) {
+        const float* x = In + e * nin;
+        float v = 0.f;
+        for (int t = t0; t < t1; ++t) {
+          const int2 tm = s_term[t];
+          v = fmaf(__int_as_float(tm.y), x[tm.x], v);
+        }
+        out[(g0 + e) * nout + q] = v;
       }
-      blocks[(g0 + e) * nb + q] = v;
     }
   }
 }
 
-// Block -> label: one thread per label of `te` blocks staged per CTA.
-__global__ void __launch_bounds__(256) blocks_to_labels_kernel(const float* __restrict__ blocks, long long n,
-                                                               const __grid_constant__ LabelTables T, int te,
-                                                               float* __restrict__ labels) {
-  extern __shared__ float bsm[];   // [te][n_orb * n_orb]
-  const int nlab = T.n_lab, norb = T.n_orb, nb = norb * norb;
-  for (long long g0 = (long long)blockIdx.x * te; g0 < n; g0 += (long long)gridDim.x * te) {
-    const int ne = (int)min((long long)te, n - g0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < ne * nb; i += blockDim.x) bsm[i] = blocks[g0 * nb + i];
-    __syncthreads();
-    for (int i = threadIdx.x; i < ne * nlab; i += blockDim.x) {
-      const int e = i / nlab;
-      int q = i - e * nlab, L = 0;
-      while (q >= (2 * L + 1) * T.mult[L]) {
-        q -= (2 * L + 1) * T.mult[L];
-        ++L;
-      }
-      const int mult = T.mult[L], M = q / mult, k = q - M * mult;
-      const int ab = T.pair[L * 256 + k], a = ab >> 4, b = ab & 15;
-      const int la = T.shell_l[a], lb = T.shell_l[b], na = 2 * la + 1, nbb = 2 * lb + 1;
-      const float* c = T.cg + T.cg_off[(la * 4 + lb) * 8 + L] + M;
-      const float* h = bsm + e * nb + T.shell_off[a] * norb + T.shell_off[b];
-      float v = 0.f;
-      for (int ia = 0; ia < na; ++ia)
-        for (int jb = 0; jb < nbb; ++jb) v = fmaf(c[(ia * nbb + jb) * (2 * L + 1)], h[ia * norb + jb], v);
-      labels[(g0 + e) * nlab + (i - e * nlab)] = v;
-    }
-  }
-}
-
-int pick_te(int per_item_floats, int per_item_work) {
-  int te = 1;
-  while (te < 64 && (te * 2) * per_item_floats * 4 <= 48 * 1024 && te * per_item_work < 1024) te *= 2;
-  return te;
+cudaError_t launch_terms(const float* in, int nin, long long n, const int* ptr, const int2* term, int nout,
+                         int nterm, float* out, cudaStream_t st) {
+  size_t tab = 4 * (size_t)((nout + 2) & ~1) + 8 * (size_t)nterm;
+  const int staged = tab <= 64 * 1024 ? 1 : 0;
+  if (!staged) tab = 0;
+  int te = 32;
+  while (te > 1 && tab + (size_t)te * nin * 4 > 100 * 1024) te >>= 1;
+  const size_t sm = tab + (size_t)te * nin * 4;
+  cudaError_t err = cudaFuncSetAttribute(apply_terms_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (err != cudaSuccess) return err;
+  const long long groups = (n + te - 1) / te;
+  const int grid = (int)(groups < 148 * 2 ? groups : 148 * 2);
+  apply_terms_kernel<<<grid, 256, sm, st>>>(in, nin, n, ptr, term, nout, nterm, staged, te, out);
+  return cudaGetLastError();
 }
 
 // ---- assembly ----
@@ -300,11 +319,7 @@ extern "C" egnn_status egnn_labels_to_blocks(const float* labels, int64_t n, con
   LabelTables T;
   egnn_status s = make_tables(shell_l, n_shells, T, workspace, ws_bytes, st);
   if (s != EGNN_OK || n == 0) return s;
-  const int te = pick_te(T.n_lab, T.n_orb * T.n_orb);
-  const long long groups = (n + te - 1) / te;
-  const int grid = (int)(groups < 148 * 16 ? groups : 148 * 16);
-  labels_to_blocks_kernel<<<grid, 256, (size_t)te * T.n_lab * 4, st>>>(labels, n, T, te, blocks);
-  EGNN_CUDA_TRY(cudaGetLastError());
+  EGNN_CUDA_TRY(launch_terms(labels, T.n_lab, n, T.b_ptr, T.b_term, T.n_orb * T.n_orb, T.n_term, blocks, st));
   return EGNN_OK;
 }
 
@@ -316,11 +331,7 @@ extern "C" egnn_status egnn_blocks_to_labels(const float* blocks, int64_t n, con
   LabelTables T;
   egnn_status s = make_tables(shell_l, n_shells, T, workspace, ws_bytes, st);
   if (s != EGNN_OK || n == 0) return s;
-  const int te = pick_te(T.n_orb * T.n_orb, T.n_lab);
-  const long long groups = (n + te - 1) / te;
-  const int grid = (int)(groups < 148 * 16 ? groups : 148 * 16);
-  blocks_to_labels_kernel<<<grid, 256, (size_t)te * T.n_orb * T.n_orb * 4, st>>>(blocks, n, T, te, labels);
-  EGNN_CUDA_TRY(cudaGetLastError());
+  EGNN_CUDA_TRY(launch_terms(blocks, T.n_orb * T.n_orb, n, T.l_ptr, T.l_term, T.n_lab, T.n_term, labels, st));
   return EGNN_OK;
 }
 

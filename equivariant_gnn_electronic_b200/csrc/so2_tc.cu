@@ -1,4 +1,6 @@
-// Tensor-core (tcgen05) eSCN layer for bf16 embeddings, C = 128, mmax <= 2, lmax <= 6.
+// Tensor-core (tcgen05) eSCN building blocks for bf16 embeddings, C = 128, mmax <= 2,
+// lmax <= 6: the A-operand producer shared by the layer and the Hamiltonian head, and the
+// head's SO(2) GEMM and label / block kernels.
 //
 // Method: "MALOQ: Massively Accelerated Learning of Operators for Quantum
 // Transport", Sections II-B1 and III (rotate each edge onto one axis so the
@@ -11,25 +13,23 @@
 // here the contractions that are GEMMs run on tcgen05 and the small per-edge
 // rotations stay on the CUDA cores that feed them.
 //
-// Launches per layer (C = 128, bf16 storage and MMA operands, fp32 accumulation):
+// Launches (C = 128, bf16 storage and MMA operands, fp32 accumulation):
 //   prep_weights  packs the gate and SO(2) weight matrices into the exact
 //                 shared-memory image of K-major 128-byte-swizzled B tiles, one
 //                 tile per (pass, 64-wide K chunk), so one 1-D bulk copy moves it
 //                 (head: the label maps U^L are folded into the SO(2) rows here);
 //   Then per range of at most 4096 edge tiles (128 edges each):
-//   gate          g_e = W2 SiLU(W1 rho(|r_e|) + b1) + b2 on tcgen05 (hidden layer on
-//                 the CUDA cores), bf16 per edge;
-//   rotate        x_e = g_e * (D^l(R_e) [n_s || n_d]) for the kept rows |m| <= mmax,
+//   gate_rotate   g_e = W2 SiLU(W1 rho(|r_e|) + b1) + b2 on tcgen05 (hidden layer on
+//                 the CUDA cores), kept in shared memory, and
+//                 x_e = g_e * (D^l(R_e) [n_s || n_d]) for the kept rows |m| <= mmax,
 //                 written as ready-made A tiles;
-//   so2_gemm      D[128 x N <= 256] = A[128 x K] B[N x K]^T per pass in one of two
+//   consumer      the fused layer kernel (so2_fused.cu), or for the head so2_gemm:
+//                 D[128 x N <= 256] = A[128 x K] B[N x K]^T per pass in one of two
 //                 alternating TMEM accumulators, with B = W0 (|m| = 0) or
 //                 [W_b1 ; W_b2] read by four MMAs, one with the negate-B bit, per K
 //                 block (|m| = b > 0); the epilogue writes y_e (y0 in fp32, |m| > 0
-//                 in bf16) or, for the head, edge-frame labels (with
-//                 kTcLogitsInEpilogue it also forms the attention logits).
-//   Then logits (a_e = A SiLU(y0_e) + bA, warp per edge) and agg (one CTA per
-//   destination atom: softmax over its incoming edges, rotate back with the kept
-//   rows of D^l, weighted sum, residual; no atomics).
+//                 in bf16) or edge-frame labels;
+//   head_label / head_blocks   rotate back and form the orbital blocks.
 #include <math.h>
 
 #include "common.cuh"
@@ -39,319 +39,51 @@
 
 namespace {
 
-constexpr int kSB = 2;                 // gate kernel B stages
 constexpr int kAStage = 128 * 128;     // one 128 x 64 bf16 A tile (16 KB)
-constexpr int kBStage = 256 * 128;     // one <= 256 x 64 bf16 B tile (32 KB)
 constexpr int kTmemCols = 512;
-constexpr int kHStage = 2 * kAStage;   // radial hidden layer of a tile, K = C = 128: two A tiles
-constexpr int kPW = 8;                 // gate kernel: warps computing the hidden layer
-constexpr int kProducers = kPW * 32;
-constexpr int kThreads = (2 + kPW + 4) * 32;   // 0 loader, 1 MMA, hidden layer, 4 epilogue warps
-
-struct GateCtl {
-  uint64_t b_full[kSB], b_empty[kSB], acc_full[2], acc_empty[2];
-  uint64_t hid_full[2], hid_empty[2], mma_done;
-  uint32_t tmem_base;
-  int abort;
-};
 
 using tc::pack2;
 using tc::unpack8;
 
-// Epilogue store of one 32-column group of a pass, cooperative over a warp that owns
-// 32 consecutive TMEM lanes (rows).  Each thread stages its row's 32 values in the
-// warp's shared-memory tile (row stride 36 floats: 16-byte aligned, conflict-free for
-// both the row-wise writes and the column-wise reads); the warp then writes 4 rows
+// Epilogue store of one 32-column group of a head SO(2) pass, cooperative over a warp
+// that owns 32 consecutive TMEM lanes (edges).  Each thread stages its row's 32 values
+// in the warp's shared-memory tile (row stride 36 floats: 16-byte aligned, conflict-free
+// for both the row-wise writes and the column-wise reads); the warp then writes 4 rows
 // per instruction, each row's 32 columns contiguous, so every store covers whole
-// 128-byte (fp32) or 64-byte (16-bit) segments instead of 32 scattered pieces.
-// Gate passes add b2 and write bf16 gates; SO(2) passes write y (y0 in fp32, the
-// |m| > 0 blocks in bf16) or, in label mode, the fp32 label record.
+// 128-byte (fp32) or 64-byte (bf16) segments instead of 32 scattered pieces.  The
+// record is y (y0 in fp32, the |m| > 0 blocks in bf16) or, in label mode, fp32 labels.
 constexpr int kStageFloats = 32 * 36;   // per warp
-__device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& ps, float* st, long long e0,
-                                               long long grow0, int g, const uint32_t* ru) {
+__device__ __forceinline__ void epi_store_warp(const TcParams& P, const TcPass& ps, float* st, long long e0, int g,
+                                               const uint32_t* ru) {
   const int lane = threadIdx.x & 31;
   int col = ps.n_off + g;
-  if (ps.kind == 1 && ps.block > 0 && !P.label_mode && g >= ps.np)
-    col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
+  if (ps.block > 0 && !P.label_mode && g >= ps.np) col = (P.L - ps.block) * P.C + ps.n_off + (g - ps.np);   // y-
   float4* srow = reinterpret_cast<float4*>(st + lane * 36);
-  // gate passes: the group's 32 b2 values (bf16, 64 bytes, 16-byte aligned), all
-  // loaded through the read-only path before any store
-  uint32_t bw[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) bw[k] = 0u;
-  if (ps.kind == 0) {
-    const uint4* bp = reinterpret_cast<const uint4*>(P.b2 + col);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 w = __ldg(bp + k);
-      bw[4 * k] = w.x;
-      bw[4 * k + 1] = w.y;
-      bw[4 * k + 2] = w.z;
-      bw[4 * k + 3] = w.w;
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    float4 x = make_float4(__uint_as_float(ru[4 * q]), __uint_as_float(ru[4 * q + 1]),
-                           __uint_as_float(ru[4 * q + 2]), __uint_as_float(ru[4 * q + 3]));
-    if (ps.kind == 0) {   // bf16 pair (lo, hi) -> fp32 by placing each in the high half
-      x.x += __uint_as_float(bw[2 * q] << 16);
-      x.y += __uint_as_float(bw[2 * q] & 0xffff0000u);
-      x.z += __uint_as_float(bw[2 * q + 1] << 16);
-      x.w += __uint_as_float(bw[2 * q + 1] & 0xffff0000u);
-    }
-    srow[q] = x;
-  }
+  for (int q = 0; q < 8; ++q)
+    srow[q] = make_float4(__uint_as_float(ru[4 * q]), __uint_as_float(ru[4 * q + 1]),
+                          __uint_as_float(ru[4 * q + 2]), __uint_as_float(ru[4 * q + 3]));
   __syncwarp();
   const int c4 = (lane & 7) * 4, rs = lane >> 3;
 #pragma unroll
   for (int r0 = 0; r0 < 32; r0 += 4) {
     const int rr = r0 + rs;
     const float4 x = *reinterpret_cast<const float4*>(st + rr * 36 + c4);
-    if (ps.kind == 0) {
-      __nv_bfloat16* dst = P.gates + (grow0 + rr) * P.gcols + col + c4;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
-    } else {
-      const long long e = e0 + rr;
-      if (e < P.n_edges) {
-        uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
-        if (P.label_mode) {
-          *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + ps.roff + g + c4) = x;
-        } else if (ps.block == 0) {
-          *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + col + c4) = x;
-        } else {
-          __nv_bfloat16* dst =
-              reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) + (P.ybase[ps.block] - P.ybase[1]) + col + c4;
-          *reinterpret_cast<uint2*>(dst) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
-        }
+    const long long e = e0 + rr;
+    if (e < P.n_edges) {
+      uint8_t* yrow = P.Y + e * (long long)P.y_row_bytes;
+      if (P.label_mode) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + ps.roff + g + c4) = x;
+      } else if (ps.block == 0) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(yrow) + col + c4) = x;
+      } else {
+        __nv_bfloat16* dst =
+            reinterpret_cast<__nv_bfloat16*>(yrow + P.y0_bytes) + (P.ybase[ps.block] - P.ybase[1]) + col + c4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
       }
     }
   }
   __syncwarp();
-}
-
-
-// Radial gate GEMM, persistent over the tiles of a range: per 128-edge tile the
-// hidden layer h = SiLU(W1 rho(|r_e|) + b1) (K Gaussians) is computed on the CUDA
-// cores from W1 staged in shared memory and written as two 128 x 64 bf16 A tiles; the
-// gate passes g = h W2^T (+ b2 in the epilogue) run on tcgen05 into two 256-column
-// TMEM accumulators used alternately, so one pass drains while the next accumulates.
-// Gates are written per edge in bf16.  Warp 0 bulk-copies W2 tiles, warp 1 issues
-// the MMAs and owns TMEM, warps 2-9 compute the hidden layer (8 lanes per 128-byte row
-// slice, 4 rows per thread), warps 10-13 drain (thread = TMEM lane = edge).
-__global__ void __launch_bounds__(kThreads, 1) gate_kernel(const __grid_constant__ TcParams P) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_u32 = tc::smem_u32(smem_raw);
-  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
-  uint8_t* base = smem_raw + (base_u32 - raw_u32);
-  uint8_t* Hbuf = base + kSB * kBStage;
-  float* W1s = reinterpret_cast<float*>(Hbuf + 2 * kHStage);   // [K][C] fp32 (after two hidden buffers)
-  float* Stg = W1s + P.K * P.C;                              // epilogue staging, 4 warps
-  GateCtl* ctl = reinterpret_cast<GateCtl*>(Stg + 4 * kStageFloats);
-  const uint32_t B_u32 = base_u32;
-  const uint32_t H_u32 = base_u32 + kSB * kBStage;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  volatile int* abort = &ctl->abort;
-  const int C = P.C, K = P.K;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kSB; ++i) {
-      tc::mbar_init(tc::smem_u32(&ctl->b_full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&ctl->b_empty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(tc::smem_u32(&ctl->acc_full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&ctl->acc_empty[i]), 128);
-    }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(tc::smem_u32(&ctl->hid_full[i]), kProducers);
-      tc::mbar_init(tc::smem_u32(&ctl->hid_empty[i]), 1);
-    }
-    tc::mbar_init(tc::smem_u32(&ctl->mma_done), 1);
-    ctl->abort = 0;
-    tc::fence_barrier_init();
-  }
-  for (int i = threadIdx.x; i < C * K; i += blockDim.x) {
-    const int c = i / K, k = i - c * K;
-    W1s[k * C + c] = __bfloat162float(P.W1[i]);
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(tc::smem_u32(&ctl->tmem_base), kTmemCols);
-    tc::tmem_relinquish();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = ctl->tmem_base;
-  const long long E = P.n_edges;
-
-  if (warp == 0) {
-    // ---------------- W2 tile loader ----------------
-    if (lane == 0) {
-      uint32_t ib = 0;
-      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
-        for (int p = 0; p < P.npass && !*abort; ++p) {
-          const TcPass& ps = P.pass[p];
-          const uint32_t bytes = (uint32_t)ps.n * 128u;
-          for (int j = 0; j < ps.nk; ++j, ++ib) {
-            const int sb = ib % kSB;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_empty[sb]), ((ib / kSB) & 1) ^ 1, P.status, abort, 64)) break;
-            tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->b_full[sb]), bytes);
-            tc::bulk_g2s(B_u32 + sb * kBStage, P.wprep + ps.boff + (long long)j * bytes, bytes,
-                         tc::smem_u32(&ctl->b_full[sb]));
-          }
-        }
-      }
-      // the newest phase of each stage must have landed before the CTA exits
-      for (uint32_t k = (ib > (uint32_t)kSB ? ib - kSB : 0); k < ib; ++k) {
-        const uint32_t bar = tc::smem_u32(&ctl->b_full[k % kSB]);
-        const uint64_t t0 = tc::globaltimer();
-        while (!tc::mbar_try_wait(bar, (k / kSB) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      uint32_t ib = 0, ip = 0, it = 0;
-      for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-        const int hb = it & 1;
-        if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_full[hb]), (it >> 1) & 1, P.status, abort, 32)) break;
-        for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
-          const TcPass& ps = P.pass[p];
-          const int buf = ip & 1;
-          if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_empty[buf]), ((ip >> 1) & 1) ^ 1, P.status, abort)) break;
-          tc::tc_fence_after();
-          for (int j = 0; j < ps.nk; ++j, ++ib) {
-            const int sb = ib % kSB;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->b_full[sb]), (ib / kSB) & 1, P.status, abort)) break;
-            tc::tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = tc::sw128_desc(H_u32 + hb * kHStage + j * kAStage + ks * 32);
-              const uint64_t bd = tc::sw128_desc(B_u32 + sb * kBStage + ks * 32);
-              tc::mma_bf16(tmem + buf * 256, ad, bd, tc::idesc_bf16(128, ps.n), (j > 0 || ks > 0) ? 1u : 0u);
-            }
-            tc::mma_commit(tc::smem_u32(&ctl->b_empty[sb]));
-          }
-          tc::mma_commit(tc::smem_u32(&ctl->acc_full[buf]));
-        }
-        tc::mma_commit(tc::smem_u32(&ctl->hid_empty[hb]));
-      }
-      // every issued MMA must finish before TMEM is released
-      tc::mma_commit(tc::smem_u32(&ctl->mma_done));
-      const uint64_t t0 = tc::globaltimer();
-      while (!tc::mbar_try_wait(tc::smem_u32(&ctl->mma_done), 0) && tc::globaltimer() - t0 < 2000000000ull) {
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 2 && warp < 2 + kPW) {
-    // ---------------- hidden layer ----------------
-    const int pidx = (warp - 2) * 32 + lane;
-    const int q = pidx & 7;                    // 16-byte piece (8 channels) of a 64-channel slice
-    const int rb = pidx >> 3;                  // 0..31
-    const float mu_step = P.rcut / (float)(K - 1);
-    const float inv2s2 = 1.0f / (2.0f * mu_step * mu_step);
-    float b1v[2][8];
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) b1v[j][i] = __bfloat162float(P.b1[j * 64 + q * 8 + i]);
-    uint32_t it = 0;
-    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x, ++it) {
-      const int hb = it & 1;
-      uint8_t* Hb = Hbuf + hb * kHStage;
-      if (!tc::mbar_wait(tc::smem_u32(&ctl->hid_empty[hb]), ((it >> 1) & 1) ^ 1, P.status, abort, 64)) break;
-#pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
-        const int r = rb + 32 * u;
-        const long long e = (long long)t * 128 + r;
-        float v[2][8];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[j][i] = 0.f;
-        if (e < E) {
-          const float di = P.dist[e];
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[j][i] = b1v[j][i];
-          for (int k = 0; k < K; ++k) {
-            const float dd = di - k * mu_step;
-            const float rho = __expf(-dd * dd * inv2s2);
-            const float4* w = reinterpret_cast<const float4*>(W1s + k * C + q * 8);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const float4 w0 = w[j * 16], w1 = w[j * 16 + 1];
-              v[j][0] += w0.x * rho;
-              v[j][1] += w0.y * rho;
-              v[j][2] += w0.z * rho;
-              v[j][3] += w0.w * rho;
-              v[j][4] += w1.x * rho;
-              v[j][5] += w1.y * rho;
-              v[j][6] += w1.z * rho;
-              v[j][7] += w1.w * rho;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[j][i] = v[j][i] / (1.0f + __expf(-v[j][i]));
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint4 w;
-          w.x = pack2(v[j][0], v[j][1]);
-          w.y = pack2(v[j][2], v[j][3]);
-          w.z = pack2(v[j][4], v[j][5]);
-          w.w = pack2(v[j][6], v[j][7]);
-          *reinterpret_cast<uint4*>(Hb + j * kAStage + r * 128 + ((q ^ (r & 7)) << 4)) = w;
-        }
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(tc::smem_u32(&ctl->hid_full[hb]));
-    }
-  } else {
-    // ---------------- epilogue: thread = TMEM lane = edge ----------------
-    const int sub = warp & 3;
-    const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
-    float* st = Stg + sub * kStageFloats;
-    uint32_t ip = 0;
-    for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
-      const long long grow0 = (long long)(t - P.t_begin) * 128 + sub * 32;
-      for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
-        const TcPass& ps = P.pass[p];
-        const int buf = ip & 1;
-        if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), (ip >> 1) & 1, P.status, abort, 64)) break;
-        tc::tc_fence_after();
-        // the TMEM load of the next 32 columns is in flight while the current ones are stored
-        const uint32_t tb = tl + buf * 256;
-        uint32_t ra[32], rb[32];
-        tc::tmem_ld32_issue(tb, ra);
-        tc::tmem_ld_wait(ra);
-        for (int g = 0; g < ps.n; g += 64) {
-          const bool h1 = g + 32 < ps.n, h2 = g + 64 < ps.n;
-          if (h1) tc::tmem_ld32_issue(tb + g + 32, rb);
-          epi_store_warp(P, ps, st, 0, grow0, g, ra);
-          if (h1) {
-            tc::tmem_ld_wait(rb);
-            if (h2) tc::tmem_ld32_issue(tb + g + 64, ra);
-            epi_store_warp(P, ps, st, 0, grow0, g + 32, rb);
-            if (h2) tc::tmem_ld_wait(ra);
-          }
-        }
-        tc::tc_fence_before();
-        tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
-      }
-    }
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, kTmemCols);
-  }
 }
 
 // One thread per element of the prepared weight image.
@@ -411,155 +143,6 @@ __global__ void prep_weights_kernel(const __grid_constant__ TcParams P, const __
   }
   // bf16 weights are copied exactly; label rows (U^L folded in, fp32 sums) round once
   reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-}
-
-// Compile-time layout of kept row r = (l, m) (rows ordered by l, then m = -min(l,MM)..):
-// its degree, its padded offset among an edge's staged Wigner rows, and (C = 128) its
-// column in y: inside the fp32 y0 section for m = 0, inside the bf16 section otherwise.
-template <int MM>
-__host__ __device__ constexpr int agg_row_l(int r) {
-  int l = 0;
-  while (r >= 2 * (l < MM ? l : MM) + 1) { r -= 2 * (l < MM ? l : MM) + 1; ++l; }
-  return l;
-}
-template <int MM>
-__host__ __device__ constexpr int agg_row_m(int r) {
-  int l = 0;
-  while (r >= 2 * (l < MM ? l : MM) + 1) { r -= 2 * (l < MM ? l : MM) + 1; ++l; }
-  return r - (l < MM ? l : MM);
-}
-template <int MM>
-__host__ __device__ constexpr int agg_po(int r) {
-  int o = 0;
-  for (int q = 0; q < r; ++q) o += ((2 * agg_row_l<MM>(q) + 1) + 3) & ~3;
-  return o;
-}
-template <int L, int MM>
-__host__ __device__ constexpr int agg_col(int r) {
-  const int l = agg_row_l<MM>(r);
-  const int ml = l < MM ? l : MM;
-  int rr = r;
-  for (int q = 0; q < l; ++q) rr -= 2 * (q < MM ? q : MM) + 1;
-  const int m = rr - ml;
-  const int b = m < 0 ? -m : m;
-  const int base16 = b <= 1 ? 0 : 2 * (L - 1) * 128;   // |m| = b block inside the bf16 section
-  return b == 0 ? l * 128 : base16 + (m > 0 ? 0 : (L - b) * 128) + (l - b) * 128;
-}
-
-// Aggregation: one CTA of 128 threads per destination atom, thread = channel.
-// Softmax statistics per head from the logits the SO(2) kernel wrote; then the
-// incoming edges in batches of kAggB whose Wigner rows and softmax weights are
-// staged in shared memory (one flat, fully parallel copy); per edge all y loads of
-// the thread's channel are issued before the FMAs.  No atomics: one owner per atom.
-constexpr int kAggB = 8;
-constexpr int kAggWfl = 236;   // >= egnn_wigner_floats(6, 2) = 235
-
-template <int MM>
-__host__ __device__ constexpr int agg_wo(int r) {   // Wigner float offset of kept row r
-  int o = 0;
-  for (int q = 0; q < r; ++q) o += 2 * agg_row_l<MM>(q) + 1;
-  return o;
-}
-
-template <int LM, int MM>
-__global__ void __launch_bounds__(128) agg_kernel(const __grid_constant__ TcParams P) {
-  constexpr int L = LM + 1;
-  constexpr int NR = (MM == 0) ? L : (MM == 1 ? 3 * L - 2 : 5 * L - 6);   // kept rows
-  __shared__ float Ds[kAggB * kAggWfl];
-  __shared__ float ps[kAggB * 16];
-  __shared__ float hmx[16], hinv[16];
-  const int d = blockIdx.x;
-  const int c = threadIdx.x;
-  const int C = P.C, H = P.H, hc = P.C / P.H;
-  const int h = c / hc;
-  int e0 = P.row_ptr[d], e1 = P.row_ptr[d + 1];
-  if (e0 < 0 || e1 < e0 || e1 > P.n_edges) {
-    if (c == 0) egnn_flag(P.status, EGNN_DEV_BAD_GRAPH);
-    e1 = e0;
-  }
-  float mx = -INFINITY;
-  for (int e = e0; e < e1; ++e) mx = fmaxf(mx, P.logits[(long long)e * H + h]);
-  float sum = 0.f;
-  for (int e = e0; e < e1; ++e) sum += __expf(P.logits[(long long)e * H + h] - mx);
-  if (c % hc == 0) {
-    hmx[h] = mx;
-    hinv[h] = e1 > e0 ? 1.0f / sum : 0.f;
-  }
-  float acc[L * L];
-#pragma unroll
-  for (int i = 0; i < L * L; ++i) acc[i] = 0.f;
-  for (int eb = e0; eb < e1; eb += kAggB) {
-    const int nb = min(kAggB, e1 - eb);
-    __syncthreads();
-    for (int i = c; i < nb * P.wfl; i += 128) {
-      const int j = i / P.wfl;
-      Ds[j * kAggWfl + (i - j * P.wfl)] = P.wig[(long long)eb * P.wfl + i];
-    }
-    for (int i = c; i < nb * H; i += 128) {
-      const int j = i / H, hh = i - j * H;
-      ps[j * 16 + hh] = __expf(P.logits[(long long)(eb + j) * H + hh] - hmx[hh]) * hinv[hh];
-    }
-    __syncthreads();
-    for (int j = 0; j < nb; ++j) {
-      const uint8_t* yrow = P.Y + (long long)(eb + j) * P.y_row_bytes;
-      const float* y32 = reinterpret_cast<const float*>(yrow) + c;
-      const __nv_bfloat16* y16 = reinterpret_cast<const __nv_bfloat16*>(yrow + P.y0_bytes) + c;
-      float yv[NR];
-      {
-        int r = 0, c16 = 0;
-#pragma unroll
-        for (int l = 0; l < L; ++l) {
-          const int ml = l < MM ? l : MM;
-#pragma unroll
-          for (int m = -ml; m <= ml; ++m, ++r) {
-            if (m == 0) {
-              yv[r] = y32[l * 128];
-            } else {
-              const int b = m < 0 ? -m : m;
-              const int col = (b == 1 ? 0 : 2 * (L - 1) * 128) + (m > 0 ? 0 : (L - b) * 128) + (l - b) * 128;
-              yv[r] = __bfloat162float(y16[col]);
-            }
-          }
-        }
-        (void)c16;
-      }
-      const float pe = ps[j * 16 + h];
-      const float* Dj = Ds + j * kAggWfl;
-      {
-        int r = 0, wo = 0;
-#pragma unroll
-        for (int l = 0; l < L; ++l) {
-          const int ml = l < MM ? l : MM;
-#pragma unroll
-          for (int m = -ml; m <= ml; ++m, ++r) {
-            const float v = pe * yv[r];
-#pragma unroll
-            for (int mp = 0; mp < 2 * l + 1; ++mp) acc[l * l + mp] += Dj[wo + mp] * v;
-            wo += 2 * l + 1;
-          }
-        }
-      }
-    }
-  }
-  const long long ob = (long long)d * L * L * C;
-#pragma unroll
-  for (int i = 0; i < L * L; ++i) {
-    const float v = __bfloat162float(P.node_in[ob + i * C + c]) + acc[i];
-    P.node_out[ob + i * C + c] = __float2bfloat16_rn(v);
-  }
-}
-
-template <int MM>
-cudaError_t launch_agg_mm(const TcParams& P, cudaStream_t st) {
-  switch (P.lmax) {
-    case 1: if (MM <= 1) agg_kernel<1, (MM <= 1 ? MM : 1)><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 2: agg_kernel<2, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 3: agg_kernel<3, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 4: agg_kernel<4, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
-    case 5: agg_kernel<5, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
-    default: agg_kernel<6, MM><<<P.n_atoms, 128, 0, st>>>(P); break;
-  }
-  return cudaGetLastError();
 }
 
 // Hamiltonian head from y.  Persistent CTAs stage U^T (all L) in shared memory once,
@@ -696,261 +279,98 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
   }
 }
 
+// 32-bit words of the staged tables of head_label_kernel, each region rounded up to a
+// multiple of four words (16 bytes); zero when the tables are read from global memory.
+struct HeadTabWords {
+  int lab, tptr, term;
+};
+__host__ __device__ inline HeadTabWords head_tab_words(int n_lab, int n_entries, int n_term, bool staged) {
+  HeadTabWords w{0, 0, 0};
+  if (staged) {
+    w.lab = (n_lab * 11 + 3) & ~3;
+    w.tptr = (n_entries + 1 + 3) & ~3;
+    w.term = (2 * n_term + 3) & ~3;
+  }
+  return w;
+}
+
 // Hamiltonian head in label mode.  The SO(2) passes already produced edge-frame labels
 // s[L, m, k] (|m| <= min(L, mmax)); per group of te edges the records and kept Wigner
 // rows are staged in shared memory, the labels are rotated back,
 // h[L, M, k] = sum_m D^L[m, M] s[L, m, k] (one thread per label), and each block entry
 // is the sum of the Clebsch-Gordan images of its shell pair's labels (one thread per
 // entry).  The rotation commutes with U^L because U^L mixes channels only.
+// Per group of te edges (persistent CTAs): records and Wigner rows staged in shared
+// memory; every label from its precomputed list of (Wigner offset, record offset) pairs;
+// every block entry from its precomputed list of (label, Clebsch-Gordan coefficient)
+// terms (both built on the host from the orbital template and the pass layout).
 __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__ TcParams P,
-                                                         const __grid_constant__ HeadTables Tb,
-                                                         float* __restrict__ blocks, int te) {
+                                                         const __grid_constant__ HeadLabelTabs Tb,
+                                                         float* __restrict__ blocks, int te, int staged) {
   extern __shared__ float hsm[];
   const int nrec = P.y_row_bytes / 4, wfl4 = (P.wfl + 3) & ~3;
-  const int nlab = Tb.n_lab, norb = Tb.n_orb, mmax = P.mmax;
-  float* Rs = hsm;                 // [te][nrec]
-  float* Ds = Rs + te * nrec;      // [te][wfl4]
-  float* Ls = Ds + te * wfl4;      // [te][nlab]
+  const int nlab = Tb.n_lab, nb = Tb.n_orb * Tb.n_orb, nterm = staged ? Tb.n_term : 0;
+  // tables staged once per CTA when small (label terms [nlab][11], entry term pointers,
+  // terms), each region starting on a 16-byte boundary (the terms are read as int2, the
+  // records behind them as float4); otherwise read through the read-only cache
+  const HeadTabWords tw = head_tab_words(nlab, nb, Tb.n_term, staged != 0);
+  int* s_lab = reinterpret_cast<int*>(hsm);
+  int* s_tptr = s_lab + tw.lab;
+  int2* s_term = reinterpret_cast<int2*>(s_tptr + tw.tptr);
+  float* Rs = reinterpret_cast<float*>(s_tptr + tw.tptr + tw.term);   // [te][nrec]
+  float* Ds = Rs + te * nrec;                              // [te][wfl4]
+  float* Ls = Ds + te * wfl4;                              // [te][nlab]
   const int tid = threadIdx.x, nt = blockDim.x;
-  __shared__ int s_mult[8], s_lab_off[8], s_woff[8], s_shell_l[16], s_shell_off[17], s_orb_shell[32];
-  __shared__ int s_cg_off[128], s_lb[3][8], s_hroff[3], s_hnr[3];
-  __shared__ int s_kidx[16 * 16 * 8];
-  for (int x = tid; x < 8; x += nt) {
-    s_mult[x] = Tb.mult[x];
-    s_lab_off[x] = Tb.lab_off[x];
-    s_woff[x] = P.woff[x];
+  if (staged) {
+    for (int i = tid; i < nlab * 11; i += nt) s_lab[i] = Tb.lab[i];
+    for (int i = tid; i <= nb; i += nt) s_tptr[i] = Tb.term_ptr[i];
+    for (int i = tid; i < nterm; i += nt) s_term[i] = Tb.term[i];
+  } else {
+    s_lab = const_cast<int*>(Tb.lab);
+    s_tptr = const_cast<int*>(Tb.term_ptr);
+    s_term = const_cast<int2*>(Tb.term);
   }
-  for (int x = tid; x < 16; x += nt) s_shell_l[x] = Tb.shell_l[x];
-  for (int x = tid; x < 17; x += nt) s_shell_off[x] = Tb.shell_off[x];
-  for (int x = tid; x < 32; x += nt) s_orb_shell[x] = Tb.orb_shell[x];
-  for (int x = tid; x < 128; x += nt) s_cg_off[x] = Tb.cg_off[x];
-  for (int x = tid; x < Tb.n_shells * Tb.n_shells * 8; x += nt) s_kidx[x] = Tb.kidx[x];
-  if (tid < 3) {
-    s_hroff[tid] = P.hroff[tid];
-    s_hnr[tid] = P.hnr[tid];
-    int acc = 0;   // offset of degree l's labels among block b's rows (l >= b)
-    for (int l = 0; l < 8; ++l) {
-      s_lb[tid][l] = acc;
-      if (l >= tid && l <= P.lmax) acc += P.mult[l];
+  const long long ngroups = (P.n_edges + te - 1) / te;
+  for (long long gi = blockIdx.x; gi < ngroups; gi += gridDim.x) {
+    const long long e0 = gi * te;
+    const int ne = (int)min((long long)te, P.n_edges - e0);
+    __syncthreads();
+    {
+      const float4* rsrc = reinterpret_cast<const float4*>(P.Y + e0 * (long long)P.y_row_bytes);
+      float4* rdst = reinterpret_cast<float4*>(Rs);
+      for (int i = tid; i < ne * nrec / 4; i += nt) rdst[i] = rsrc[i];
+      const float* wsrc = P.wig + e0 * P.wfl;
+      for (int e = 0; e < ne; ++e)
+        for (int i = tid; i < P.wfl; i += nt) Ds[e * wfl4 + i] = wsrc[(long long)e * P.wfl + i];
     }
-  }
-  const long long e0 = (long long)blockIdx.x * te;
-  const int ne = (int)min((long long)te, P.n_edges - e0);
-  {
-    const float4* rsrc = reinterpret_cast<const float4*>(P.Y + e0 * (long long)P.y_row_bytes);
-    float4* rdst = reinterpret_cast<float4*>(Rs);
-    for (int i = tid; i < ne * nrec / 4; i += nt) rdst[i] = rsrc[i];
-    const float* wsrc = P.wig + e0 * P.wfl;
-    for (int i = tid; i < ne * P.wfl; i += nt) {
-      const int e = i / P.wfl;
-      Ds[e * wfl4 + (i - e * P.wfl)] = wsrc[i];
+    __syncthreads();
+    for (int q = tid; q < nlab; q += nt) {
+      const int* lt = s_lab + q * 11;
+      const int cnt = lt[0];
+      for (int e = 0; e < ne; ++e) {
+        const float* De = Ds + e * wfl4;
+        const float* Re = Rs + e * nrec;
+        float h = 0.f;
+        for (int j = 0; j < cnt; ++j) h = fmaf(De[lt[1 + j]], Re[lt[6 + j]], h);
+        Ls[e * nlab + q] = h;
+      }
     }
-  }
-  __syncthreads();
-  for (int i = tid; i < ne * nlab; i += nt) {
-    const int e = i / nlab, q0 = i - e * nlab;
-    int q = q0, Lq = 0;
-    while (q >= (2 * Lq + 1) * s_mult[Lq]) {
-      q -= (2 * Lq + 1) * s_mult[Lq];
-      ++Lq;
-    }
-    const int mult = s_mult[Lq], M = q / mult, k = q - M * mult;
-    const int ml = Lq < mmax ? Lq : mmax, dl = 2 * Lq + 1;
-    const float* De = Ds + e * wfl4 + s_woff[Lq] + M;   // row m of D^L at (m + ml) * dl
-    const float* Re = Rs + e * nrec;
-    float h = De[ml * dl] * Re[s_hroff[0] + s_lb[0][Lq] + k];
-    for (int b = 1; b <= ml; ++b) {
-      // pass qq of block b holds label rows [R qq, R qq + npq) of s+ then of s-, R = kTcPairRows
-      const int r = s_lb[b][Lq] + k, qq = r / kTcPairRows, w = r - qq * kTcPairRows;
-      const int rest = s_hnr[b] - kTcPairRows * qq;
-      const int npq = rest >= kTcPairRows ? kTcPairRows : ((rest + 15) & ~15);
-      const int base = s_hroff[b] + 2 * kTcPairRows * qq + w;
-      h += De[(ml + b) * dl] * Re[base] + De[(ml - b) * dl] * Re[base + npq];
-    }
-    Ls[e * nlab + q0] = h;
-  }
-  __syncthreads();
-  for (int i = tid; i < ne * norb * norb; i += nt) {
-    const int e = i / (norb * norb), q = i - e * norb * norb;
-    const int ri = q / norb, cj = q - ri * norb;
-    const int a = s_orb_shell[ri], b = s_orb_shell[cj];
-    const int la = s_shell_l[a], lb = s_shell_l[b];
-    const int ia = ri - s_shell_off[a], jb = cj - s_shell_off[b];
-    float v = 0.f;
-    for (int Lc = (la > lb ? la - lb : lb - la); Lc <= la + lb; ++Lc) {
-      const int k = s_kidx[(a * Tb.n_shells + b) * 8 + Lc];
-      const float* cgm = Tb.cg + s_cg_off[(la * 4 + lb) * 8 + Lc] + (ia * (2 * lb + 1) + jb) * (2 * Lc + 1);
-      const float* h = Ls + e * nlab + s_lab_off[Lc] + k;
-      const int mult = s_mult[Lc];
-      for (int M = 0; M < 2 * Lc + 1; ++M) v += cgm[M] * h[M * mult];
-    }
-    blocks[(e0 + e) * norb * norb + q] = v;
-  }
-}
-
-
-// Attention logits a_{e,h} = A[h] . SiLU(y0_e) + bA[h], one warp per edge: lanes
-// read y0 (fp32, coalesced) and A from shared memory, stored column-major with a
-// column's heads contiguous (stride HS = 4 ceil(H/4) + 4 floats: 16-byte aligned and
-// free of bank conflicts for eight lanes' 16-byte reads), so one 16-byte read serves
-// four heads; the next edge's y0 is loaded while this edge is reduced; the heads'
-// partial sums are then reduced across the warp.
-__global__ void __launch_bounds__(256) logits_kernel(const __grid_constant__ TcParams P) {
-  extern __shared__ float As[];                 // [L*C][HS]
-  const int LC = P.L * P.C, H = P.H, HQ = (H + 3) >> 2, HS = 4 * HQ + 4;
-  for (int i = threadIdx.x; i < LC * HS; i += blockDim.x) {
-    const int j = i / HS, h = i - j * HS;
-    As[i] = h < H ? P.Af[h * LC + j] : 0.f;
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
-  long long e = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  float yv[28];                                  // LC <= 7 * 128 = 896 = 28 * 32
-  if (e < P.n_edges) {
-    const float* y0 = reinterpret_cast<const float*>(P.Y + e * (long long)P.y_row_bytes);
-#pragma unroll
-    for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
-  }
-  for (; e < P.n_edges; e += nw) {
-    float a[16];
-#pragma unroll
-    for (int h = 0; h < 16; ++h) a[h] = 0.f;
-#pragma unroll
-    for (int k = 0; k < 28; ++k) {
-      const int j = lane + 32 * k;
-      if (j < LC) {
-        const float sv = yv[k] / (1.0f + __expf(-yv[k]));
-        const float4* ap = reinterpret_cast<const float4*>(As + j * HS);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (q < HQ) {
-            const float4 w = ap[q];
-            a[4 * q] += w.x * sv;
-            a[4 * q + 1] += w.y * sv;
-            a[4 * q + 2] += w.z * sv;
-            a[4 * q + 3] += w.w * sv;
-          }
+    __syncthreads();
+    for (int q = tid; q < nb; q += nt) {
+      const int t0 = s_tptr[q], t1 = s_tptr[q + 1];
+      for (int e = 0; e < ne; ++e) {
+        const float* Le = Ls + e * nlab;
+        float v = 0.f;
+        for (int t = t0; t < t1; ++t) {
+          const int2 tm = s_term[t];
+          v = fmaf(__int_as_float(tm.y), Le[tm.x], v);
         }
-      }
-    }
-    const long long en = e + nw;
-    if (en < P.n_edges) {
-      const float* y0 = reinterpret_cast<const float*>(P.Y + en * (long long)P.y_row_bytes);
-#pragma unroll
-      for (int k = 0; k < 28; ++k) yv[k] = (lane + 32 * k < LC) ? y0[lane + 32 * k] : 0.f;
-    }
-#pragma unroll
-    for (int h = 0; h < 16; ++h) {
-      if (h < H) {
-        float x = a[h];
-#pragma unroll
-        for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        if (lane == 0) P.logits[e * H + h] = x + __bfloat162float(P.bA[h]);
+        blocks[(e0 + e) * nb + q] = v;
       }
     }
   }
 }
 
-// ---------------- rotate + gate: the A operands of the SO(2) GEMM ----------------
-// One CTA per 128-edge tile.  For every edge and degree l the kept rows of the edge
-// frame, x[l, m, :] = g[l, :] * sum_{m'} D^l[m, m'] [n_s || n_d][l, m', :] for
-// |m| <= min(l, mmax), are accumulated in fp32 (packed two-wide FMAs) from the bf16
-// node table, multiplied by the gates in fp32 and rounded once to the bf16 MMA operand,
-// then written straight into the 128-byte-swizzled K-major 128 x 64 tiles that the
-// GEMM's bulk copies move (16-byte piece c of row r at position c ^ (r & 7)).
-// Warp = one edge at a time, lane = one 8-channel piece of the 256-wide pair row
-// (lanes 0-15 the source atom, 16-31 the destination): a node row is one 512-byte
-// warp load, an A row four full 128-byte lines.  All 2l+1 rows of n[l] are loaded
-// before the FMAs, which keeps up to 13 x 16 B per lane in flight.
-template <int LM, int MM>
-__global__ void __launch_bounds__(256) rotate_kernel(const __grid_constant__ TcParams P) {
-  constexpr int L = LM + 1;
-  __shared__ int s_node[2][128];   // source and destination atom of each row
-  const int t = P.t_begin + blockIdx.x;
-  const long long E = P.n_edges;
-  if (threadIdx.x < 128) {
-    const int r = threadIdx.x;
-    const long long e = (long long)t * 128 + r;
-    int sv = 0, dv = 0;
-    if (e < E) {
-      sv = P.src[e];
-      int lo = 0, hi = P.n_atoms;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
-      }
-      dv = lo;
-      if (sv < 0 || sv >= P.n_atoms) {
-        egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
-        sv = dv;
-      }
-    }
-    s_node[0][r] = sv;
-    s_node[1][r] = dv;
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int side = lane >> 4, cs = lane >> 3, qq = lane & 7;
-  uint8_t* xt = P.X + (long long)blockIdx.x * P.nch * 16384;
-  for (int r = warp; r < 128; r += 8) {
-    const long long e = (long long)t * 128 + r;
-    const bool valid = e < E;
-    const __nv_bfloat16* zn = P.node_in + (long long)s_node[side][r] * (L * L) * 128 + (lane & 15) * 8;
-    const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl;
-    const __nv_bfloat16* gr = P.gates + ((long long)blockIdx.x * 128 + r) * P.gcols + lane * 8;
-    uint8_t* xr = xt + r * 128 + ((qq ^ (r & 7)) << 4);
-    int wo = 0;
-#pragma unroll
-    for (int l = 0; l < L; ++l) {
-      const int dl = 2 * l + 1, ml = l < MM ? l : MM, nr = 2 * ml + 1;
-      // the nr x dl kept coefficients of D^l, spread over the lanes
-      float cf[3];
-#pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        const int idx = lane + 32 * k;
-        cf[k] = (valid && idx < nr * dl) ? __ldg(De + wo + idx) : 0.f;
-      }
-      uint4 zq[2 * LM + 1];
-#pragma unroll
-      for (int mp = 0; mp < dl; ++mp)
-        zq[mp] = valid ? __ldg(reinterpret_cast<const uint4*>(zn + (l * l + mp) * 128)) : make_uint4(0, 0, 0, 0);
-      const uint4 gq = valid ? __ldg(reinterpret_cast<const uint4*>(gr + l * 256)) : make_uint4(0, 0, 0, 0);
-      float2 acc[2 * MM + 1][4];
-#pragma unroll
-      for (int m = 0; m < nr; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][i] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int mp = 0; mp < dl; ++mp) {
-        float z[8];
-        unpack8(zq[mp], z);
-#pragma unroll
-        for (int m = 0; m < nr; ++m) {
-          const int k = m * dl + mp;
-          const float c = __shfl_sync(0xffffffffu, cf[k >> 5], k & 31);
-          const float2 c2 = make_float2(c, c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[m][i] = __ffma2_rn(c2, make_float2(z[2 * i], z[2 * i + 1]), acc[m][i]);
-        }
-      }
-      float g[8];
-      unpack8(gq, g);
-#pragma unroll
-      for (int m = 0; m < nr; ++m) {
-        const int mm = m - ml, b = mm < 0 ? -mm : mm;
-        const int id = b == 0 ? l * 4 + cs : P.xbase[b] + ((l - b) * 4 + cs) * 2 + (mm < 0 ? 1 : 0);
-        uint4 w;
-        w.x = pack2(acc[m][0].x * g[0], acc[m][0].y * g[1]);
-        w.y = pack2(acc[m][1].x * g[2], acc[m][1].y * g[3]);
-        w.z = pack2(acc[m][2].x * g[4], acc[m][2].y * g[5]);
-        w.w = pack2(acc[m][3].x * g[6], acc[m][3].y * g[7]);
-        *reinterpret_cast<uint4*>(xr + (long long)id * 16384) = w;
-      }
-      wo += nr * dl;
-    }
-  }
-}
 
 // ---------------- gate + rotate in one kernel: the A operands, gates kept on chip ----------------
 // Persistent over the tiles of a range (one CTA per SM).  Per 128-edge tile:
@@ -1346,7 +766,6 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const long long E = P.n_edges;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1460,15 +879,8 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
     const int r = sub * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(sub * 32) << 16);
     float* st = Stg + sub * kStageFloats;
-    const int LC = P.L * P.C, H = P.H;
-    const bool logits = kTcLogitsInEpilogue && P.with_logits && !P.label_mode;
     uint32_t ip = 0;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
-      const long long e = (long long)t * 128 + r;
-      const bool valid = e < E;
-      float la[16];   // attention logits of this edge, accumulated over the |m| = 0 passes
-#pragma unroll
-      for (int h = 0; h < 16; ++h) la[h] = 0.f;
       for (int p = 0; p < P.npass && !*abort; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
         const int buf = kNBuf == 2 ? (ip & 1) : 0;
@@ -1476,40 +888,14 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
         const uint32_t tb = tl + buf * 256;
         if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), ph, P.status, abort, 128)) break;
         tc::tc_fence_after();
-        const bool lg = logits && ps.block == 0;
         for (int g = 0; g < ps.n; g += 32) {
           uint32_t ra[32];
           tc::tmem_ld32_issue(tb + g, ra);
           tc::tmem_ld_wait(ra);
-          epi_store_warp(P, ps, st, (long long)t * 128 + sub * 32, 0, g, ra);
-          if (lg) {
-            // a_h += A[h, j] SiLU(y0_j) over this group's 32 columns j of y0
-            const float* Ag = P.Af + ps.n_off + g;
-#pragma unroll
-            for (int i4 = 0; i4 < 8; ++i4) {
-              float sv[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const float y = __uint_as_float(ra[4 * i4 + c]);
-                sv[c] = y / (1.0f + __expf(-y));
-              }
-#pragma unroll
-              for (int h = 0; h < 16; ++h) {
-                if (h < H) {
-                  const float4 a = __ldg(reinterpret_cast<const float4*>(Ag + h * LC) + i4);
-                  la[h] += a.x * sv[0] + a.y * sv[1] + a.z * sv[2] + a.w * sv[3];
-                }
-              }
-            }
-          }
+          epi_store_warp(P, ps, st, (long long)t * 128 + sub * 32, g, ra);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
-        if (lg && ps.last_of_kind && valid) {
-#pragma unroll
-          for (int h = 0; h < 16; ++h)
-            if (h < H) P.logits[e * H + h] = la[h] + __bfloat162float(P.bA[h]);
-        }
       }
     }
   }
@@ -1522,15 +908,6 @@ __global__ void __launch_bounds__(kGThreads, 1) so2_gemm_kernel(const __grid_con
 }
 
 }  // namespace
-
-size_t gate_smem_bytes(int K, int C) {
-  return kSB * kBStage + 2 * kHStage + sizeof(float) * ((size_t)K * C + 4 * kStageFloats) + sizeof(GateCtl) + 1024;
-}
-
-__global__ void a_to_f32_kernel(const __nv_bfloat16* __restrict__ A, float* __restrict__ out, int n) {
-  int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) out[i] = __bfloat162float(A[i]);
-}
 
 // Check of the bounded wait every pipelined kernel uses: one thread waits on an
 // mbarrier that nothing arrives on, with the given limit, through the same routine
@@ -1582,28 +959,6 @@ cudaError_t tc_profile_read(double* ms, long long* launches, long long* edges) {
   *launches = g_prof_n;
   *edges = g_prof_edges;
   return cudaSuccess;
-}
-
-template <int LM, int MM>
-static void launch_rotate(const TcParams& P, int nt, cudaStream_t st) {
-  rotate_kernel<LM, MM><<<nt, 256, 0, st>>>(P);
-}
-
-static cudaError_t launch_rotate_any(const TcParams& P, int nt, cudaStream_t st) {
-  switch (P.mmax * 8 + P.lmax) {
-#define EGNN_ROT_CASE(LMv, MMv) \
-  case MMv * 8 + LMv:          \
-    launch_rotate<LMv, MMv>(P, nt, st); \
-    break;
-    EGNN_ROT_CASE(1, 0) EGNN_ROT_CASE(2, 0) EGNN_ROT_CASE(3, 0) EGNN_ROT_CASE(4, 0) EGNN_ROT_CASE(5, 0)
-    EGNN_ROT_CASE(6, 0) EGNN_ROT_CASE(1, 1) EGNN_ROT_CASE(2, 1) EGNN_ROT_CASE(3, 1) EGNN_ROT_CASE(4, 1)
-    EGNN_ROT_CASE(5, 1) EGNN_ROT_CASE(6, 1) EGNN_ROT_CASE(2, 2) EGNN_ROT_CASE(3, 2) EGNN_ROT_CASE(4, 2)
-    EGNN_ROT_CASE(5, 2) EGNN_ROT_CASE(6, 2)
-#undef EGNN_ROT_CASE
-    default:
-      return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
 }
 
 static cudaError_t launch_gate_rotate_any(const TcParams& P, int grid, size_t smem, cudaStream_t st) {
@@ -1684,11 +1039,7 @@ static cudaError_t so2_gemm_consumer(const TcParams& Ps, int grid, cudaStream_t 
 }
 
 static cudaError_t launch_tc_gemm(const TcParams& P, const TcWeights& W, cudaStream_t st) {
-  if (P.with_logits) {
-    const int na = P.H * P.L * P.C;
-    a_to_f32_kernel<<<(na + 255) / 256, 256, 0, st>>>(P.A, P.Af, na);
-  }
-  return launch_tc_pipeline(P, W, st, so2_gemm_consumer, nullptr, P.with_logits && !P.label_mode);
+  return launch_tc_pipeline(P, W, st, so2_gemm_consumer, nullptr, false);
 }
 
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te) {
@@ -1696,21 +1047,26 @@ size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te) {
 }
 
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
-                           float* blocks, cudaStream_t st) {
+                           const HeadLabelTabs& LT, float* blocks, cudaStream_t st) {
   cudaError_t err = launch_tc_gemm(P, W, st);
   if (err != cudaSuccess || P.n_edges == 0) return err;
   if (P.label_mode) {
-    const int te_max = 16;
+    const int nb = LT.n_orb * LT.n_orb;
+    const HeadTabWords tw = head_tab_words(LT.n_lab, nb, LT.n_term, true);
+    size_t tab = 4 * ((size_t)tw.lab + tw.tptr + tw.term);
+    const int staged = tab <= 64 * 1024 ? 1 : 0;
+    if (!staged) tab = 0;
     auto bytes = [&](int t) {
-      return sizeof(float) * (size_t)t * (size_t)(P.y_row_bytes / 4 + ((P.wfl + 3) & ~3) + T.n_lab);
+      return tab + sizeof(float) * (size_t)t * (size_t)(P.y_row_bytes / 4 + ((P.wfl + 3) & ~3) + T.n_lab);
     };
-    int te = te_max;
-    while (te > 1 && bytes(te) > 100 * 1024) te >>= 1;
-    if (bytes(te) > 200 * 1024) return cudaErrorInvalidValue;
+    int te = 32;   // edges per group: two CTAs per SM within ~110 KB of shared memory each
+    while (te > 1 && bytes(te) > 110 * 1024) te >>= 1;
+    if (bytes(te) > 220 * 1024) return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(head_label_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes(te));
     if (err != cudaSuccess) return err;
     const long long groups = (P.n_edges + te - 1) / te;
-    head_label_kernel<<<(unsigned)groups, 256, bytes(te), st>>>(P, T, blocks, te);
+    const int grid = (int)(groups < 4LL * P.grid ? groups : 4LL * P.grid);
+    head_label_kernel<<<grid, 256, bytes(te), st>>>(P, LT, blocks, te, staged);
     return cudaGetLastError();
   }
   int u_total = 0;
@@ -1737,24 +1093,4 @@ cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTabl
       return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
-}
-
-cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st) {
-  cudaError_t err = launch_tc_gemm(P, W, st);
-  if (err != cudaSuccess) return err;
-  if (!kTcLogitsInEpilogue && P.n_edges > 0) {
-    const size_t sm = sizeof(float) * (size_t)(4 * ((P.H + 3) / 4) + 4) * P.L * P.C;
-    err = cudaFuncSetAttribute(logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (err != cudaSuccess) return err;
-    int nb = 2;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, logits_kernel, 256, sm);
-    logits_kernel<<<(nb > 0 ? nb : 1) * P.grid, 256, sm, st>>>(P);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-  }
-  switch (P.mmax) {
-    case 0: return launch_agg_mm<0>(P, st);
-    case 1: return launch_agg_mm<1>(P, st);
-    default: return launch_agg_mm<2>(P, st);
-  }
 }

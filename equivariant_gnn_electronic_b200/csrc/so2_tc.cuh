@@ -37,11 +37,8 @@ struct TcParams {
   const __nv_bfloat16 *W1, *b1, *b2, *A, *bA;
   const uint8_t* wprep;
   long long wprep_bytes;
-  uint8_t* Y;                    // [n_edges][y_row_bytes]
-  float* logits;                 // [n_edges][H]
-  float* Af;                     // attention matrix A[H][L*C] in fp32 (workspace copy)
+  uint8_t* Y;                    // head: [n_edges][y_row_bytes]
   int32_t* status;
-  int with_logits;               // 1: layer (attention logits from SiLU(y0)); 0: head
   // Label mode (head only): the SO(2) weights are pre-multiplied by the label maps U^L,
   // so a pass produces labels in the edge frame, s[l, m, k] = sum_c U^l[k, c] y[l, m, c],
   // stored in fp32 as the concatenation of the passes' accumulators (record of
@@ -51,13 +48,11 @@ struct TcParams {
   int hnr[3];                    // label rows of block b: sum_{l >= b} mult_l
   int mult[8];                   // labels per L
   const __nv_bfloat16* U[8];     // U^L [mult_L][C]
-  // Tile range of one launch and the per-range buffers of the split pipeline
-  // (gate GEMM -> rotate -> SO(2) GEMM): gates of the range's rows in bf16, and the
-  // rotated, gated A operands as 128 x 64 bf16 tiles in the 128-byte-swizzled
+  // Tile range of one launch and the per-range buffer of the pipeline (gate + rotate ->
+  // SO(2) GEMM): the rotated, gated A operands as 128 x 64 bf16 tiles in the 128-byte-swizzled
   // K-major image the MMA reads, `nch` tiles per edge tile, block b's first at
   // xbase[b] (a |m| > 0 K block stores x+ then x-).
   int t_begin, t_end;
-  __nv_bfloat16* gates;          // [(t_end - t_begin) * 128][gcols]
   uint8_t* X;                    // [(t_end - t_begin)][nch][128 * 128 B]
   int nch;
   int xbase[3];
@@ -88,16 +83,12 @@ constexpr int kTcMaxGrid = 160;
 
 // SO(2) GEMM pass width in TMEM columns: 512 = one accumulator per pass (fewer A
 // re-reads, drain between passes), 256 = two alternating accumulators (drain overlaps
-// the next pass).  Attention logits: in the GEMM epilogue (1) or a separate kernel (0).
+// the next pass).
 #ifndef EGNN_ACC_COLS
 #define EGNN_ACC_COLS 256
 #endif
-#ifndef EGNN_LOGITS_IN_EPILOGUE
-#define EGNN_LOGITS_IN_EPILOGUE 0
-#endif
 constexpr int kTcAccCols = EGNN_ACC_COLS;
 constexpr int kTcPairRows = kTcAccCols / 2;   // label / output rows per half of a |m| > 0 pass
-constexpr bool kTcLogitsInEpilogue = EGNN_LOGITS_IN_EPILOGUE != 0;
 constexpr int kTcChunkTiles = 4096;   // edge tiles per launch range (bounds the gate and A buffers)
 
 // Tiles per launch range: the fewest ranges of at most kTcChunkTiles, balanced.
@@ -111,17 +102,25 @@ struct HeadTables;
 struct HeadUPtrs {
   const __nv_bfloat16* U[8];
 };
+// Precomputed tables of the label-mode head (device memory, built on the host):
+// lab[q][11]: number of terms, then up to five Wigner offsets and five record offsets
+// of label q's rotate-back; term_ptr[n_orb^2 + 1] / term[]: per block entry its terms
+// (label index, Clebsch-Gordan coefficient as float bits).
+struct HeadLabelTabs {
+  int n_lab, n_orb, n_term;
+  const int* lab;
+  const int* term_ptr;
+  const int2* term;
+};
 
-size_t gate_smem_bytes(int K, int C);
 // Consumer of one range's A tiles: launches its kernel over tiles [Ps.t_begin, Ps.t_end).
 using TcConsumer = cudaError_t (*)(const TcParams& Ps, int grid, cudaStream_t st, void* ctx);
 cudaError_t launch_tc_pipeline(const TcParams& P, const TcWeights& W, cudaStream_t st, TcConsumer consumer,
                                void* ctx, bool profiled);
-cudaError_t launch_layer_tc(const TcParams& P, const TcWeights& W, cudaStream_t st);
 cudaError_t launch_layer_fused(const TcParams& P, const TcWeights& W, cudaStream_t st);
 size_t layer_fused_smem_bytes(int lmax, int heads);
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
-                           float* blocks, cudaStream_t st);
+                           const HeadLabelTabs& LT, float* blocks, cudaStream_t st);
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te);
 void tc_profile_enable(bool on);
 cudaError_t launch_wait_check(int32_t* status, unsigned long long limit_ns, cudaStream_t st);

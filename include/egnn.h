@@ -96,7 +96,7 @@ enum {
   EGNN_WS_BUILD_GRAPH = 0,
   EGNN_WS_LAYER = 1,
   EGNN_WS_HAMILTONIAN = 2,
-  EGNN_WS_LABELS = 3,       /* egnn_labels_to_blocks / egnn_blocks_to_labels (64 KB)  */
+  EGNN_WS_LABELS = 3,       /* egnn_labels_to_blocks / egnn_blocks_to_labels (1 MB)   */
   EGNN_WS_ASSEMBLY = 4      /* egnn_assemble_hamiltonian (4 bytes per atom)          */
 };
 

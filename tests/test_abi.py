@@ -104,7 +104,7 @@ def test_layer_workspace_stores_no_per_edge_message():
 
 
 def test_head_workspace_grows_by_the_message_record_per_edge():
-    # tensor-core head: per edge the y record (y0 fp32, |m| > 0 bf16) and the logits slot
+    # tensor-core head: per edge only the y record (y0 fp32, |m| > 0 bf16)
     L, C, H = 5, 128, 8
     d = egnn.make_desc(4, 2, C, H, 32, 8.0, "bf16")
     rec = 4 * L * C + 4 * C * ((L - 1) + (L - 2))
@@ -112,4 +112,4 @@ def test_head_workspace_grows_by_the_message_record_per_edge():
     w1 = egnn.workspace_bytes(egnn.EGNN_WS_HAMILTONIAN, d, 1000, e1)
     w2 = egnn.workspace_bytes(egnn.EGNN_WS_HAMILTONIAN, d, 1000, e2)
     per_edge = (w2 - w1) / (e2 - e1)
-    assert abs(per_edge - (rec + 4 * H)) < 1.0
+    assert abs(per_edge - rec) < 1.0

@@ -177,7 +177,7 @@ bool tc_plan(const egnn_layer_desc* d, TcParams& P, const int* mult = nullptr) {
       boff += (long long)q.n * kblocks * 128;
     }
   }
-  // A tiles of one edge tile for the split pipeline: block 0 one per (l, 64 channels),
+  // A tiles of one edge tile (gate_rotate output): block 0 one per (l, 64 channels),
   // |m| = b > 0 an x+ / x- pair per (l >= b, 64 channels)
   const int kpl = 2 * C / 64;
   P.xbase[0] = 0;

@@ -12,9 +12,10 @@
 // for the 8,064-atom GeSbTe cell.
 //
 // Kernels:
-//   apply_terms       both directions: a group of blocks (or label vectors) staged in
-//                     shared memory, one thread per output element (matrix element, or
-//                     label) summing its precomputed Clebsch-Gordan terms; the term
+//   apply_terms       both directions: groups of blocks (or label vectors) brought into
+//                     shared memory by 1-D bulk copies, the next group's copy in flight
+//                     while the current one is summed; one (item, output element) per
+//                     work item summing its precomputed Clebsch-Gordan terms; the term
 //                     lists are built on the host from the orbital template.
 //   h_count / h_scan / h_fill  block-sparse rows of the k = 0 Hamiltonian: row block d
 //                     holds the on-site block of d and, per distinct source atom s of
@@ -27,6 +28,7 @@
 
 #include "common.cuh"
 #include "so2_params.cuh"
+#include "tc_ptx.cuh"
 
 namespace {
 
@@ -127,17 +129,32 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
 }
 
 // out[item][q] = sum over the terms of q of coefficient * in[item][index], for `te` items
-// per group staged in shared memory (persistent CTAs; the term list staged once per CTA
-// when it fits).  One thread per output element q, looping over the group's items.
+// per group (persistent CTAs; the term list staged once per CTA when it fits).  Each
+// group's inputs are contiguous in global memory and arrive by one 1-D bulk copy into
+// one of two shared-memory stages, issued one group ahead; a group whose byte count is
+// not a multiple of 16 (only a ragged last group can be) is loaded by all threads
+// instead.  One (item, q) output per work item: consecutive work items are consecutive
+// outputs of the group, so the stores are contiguous.  Waits are bounded (2 s); a wait
+// that runs out ends every thread's loop at the same group.
 __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restrict__ in, int nin, long long n,
                                                           const int* __restrict__ ptr, const int2* __restrict__ term,
-                                                          int nout, int nterm, int staged, int te,
+                                                          int nout, int nterm, int staged, int te, int bulk,
                                                           float* __restrict__ out) {
-  extern __shared__ float tsm[];
+  extern __shared__ __align__(16) float tsm[];
+  __shared__ uint64_t full[2];
+  __shared__ int abort_flag;
+  const int ptr_words = staged ? ((nout + 4) & ~3) : 0;
+  const int tab_words = staged ? ptr_words + 2 * ((nterm + 1) & ~1) : 0;
   int* s_ptr = reinterpret_cast<int*>(tsm);
-  int2* s_term = reinterpret_cast<int2*>(s_ptr + (staged ? ((nout + 2) & ~1) : 0));
-  float* In = reinterpret_cast<float*>(s_term + (staged ? nterm : 0));   // [te][nin]
+  int2* s_term = reinterpret_cast<int2*>(s_ptr + ptr_words);
+  float* stage[2] = {tsm + tab_words, tsm + tab_words + te * nin};   // [te][nin] each
   const int tid = threadIdx.x, nt = blockDim.x;
+  if (tid == 0) {
+    tc::mbar_init(tc::smem_u32(&full[0]), 1);
+    tc::mbar_init(tc::smem_u32(&full[1]), 1);
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
   if (staged) {
     for (int i = tid; i <= nout; i += nt) s_ptr[i] = ptr[i];
     for (int i = tid; i < nterm; i += nt) s_term[i] = term[i];
@@ -145,21 +162,66 @@ __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restric
     s_ptr = const_cast<int*>(ptr);
     s_term = const_cast<int2*>(term);
   }
-  for (long long g0 = (long long)blockIdx.x * te; g0 < n; g0 += (long long)gridDim.x * te) {
+  __syncthreads();
+  const long long ngroups = (n + te - 1) / te;
+  // a group goes by bulk copy when its byte count is a multiple of 16
+  auto by_copy = [&](long long gi) {
+    return bulk && (((long long)min((long long)te, n - gi * te) * nin * 4) & 15) == 0;
+  };
+  auto issue = [&](long long gi, int st) {   // thread 0 only
+    const uint32_t bytes = (uint32_t)(min((long long)te, n - gi * te) * nin * 4);
+    const uint32_t bar = tc::smem_u32(&full[st]);
+    tc::mbar_arrive_expect_tx(bar, bytes);
+    tc::bulk_g2s(tc::smem_u32(stage[st]), in + gi * te * nin, bytes, bar);
+  };
+  uint32_t phase[2] = {0u, 0u};
+  bool pend[2] = {false, false};   // thread 0: a copy into the stage is in flight
+  int it = 0;
+  if (tid == 0 && blockIdx.x < ngroups && by_copy(blockIdx.x)) {
+    issue(blockIdx.x, 0);
+    pend[0] = true;
+  }
+  for (long long gi = blockIdx.x; gi < ngroups; gi += gridDim.x, ++it) {
+    const int st = it & 1;
+    const long long g0 = gi * te;
     const int ne = (int)min((long long)te, n - g0);
-    __syncthreads();
-    for (int i = tid; i < ne * nin; i += nt) In[i] = in[g0 * nin + i];
-    __syncthreads();
-    for (int q = tid; q < nout; q += nt) {
-      const int t0 = s_ptr[q], t1 = s_ptr[q + 1];
-      for (int e = 0; e < ne; ++e) {
-        const float* x = In + e * nin;
-        float v = 0.f;
-        for (int t = t0; t < t1; ++t) {
-          const int2 tm = s_term[t];
-          v = fmaf(__int_as_float(tm.y), x[tm.x], v);
-        }
-        out[(g0 + e) * nout + q] = v;
+    const long long gn = gi + gridDim.x;
+    if (tid == 0 && gn < ngroups && by_copy(gn)) {
+      issue(gn, st ^ 1);
+      pend[st ^ 1] = true;
+    }
+    float* In = stage[st];
+    if (by_copy(gi)) {
+      const bool ok = tc::mbar_wait(tc::smem_u32(&full[st]), phase[st], nullptr, &abort_flag, 0);
+      if (!__syncthreads_and(ok)) break;
+      phase[st] ^= 1u;
+      pend[st] = false;
+    } else {
+      for (int i = tid; i < ne * nin; i += nt) In[i] = in[g0 * nin + i];
+      __syncthreads();
+    }
+    int e = tid / nout, q = tid - e * nout;
+    float* o = out + g0 * nout;
+    for (int w = tid; w < ne * nout; w += nt) {
+      const float* x = In + e * nin;
+      const int t1 = s_ptr[q + 1];
+      float v = 0.f;
+      for (int t = s_ptr[q]; t < t1; ++t) {
+        const int2 tm = s_term[t];
+        v = fmaf(__int_as_float(tm.y), x[tm.x], v);
+      }
+      o[w] = v;
+      q += nt;
+      while (q >= nout) { q -= nout; ++e; }
+    }
+    __syncthreads();   // stage st is free for the copy issued in the next iteration
+  }
+  // a copy still in flight (only after a wait ran out) must land before the CTA exits
+  if (tid == 0) {
+    for (int st = 0; st < 2; ++st) {
+      if (!pend[st]) continue;
+      const uint64_t t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(tc::smem_u32(&full[st]), phase[st]) && tc::globaltimer() - t0 < 2000000000ull) {
       }
     }
   }
@@ -167,17 +229,24 @@ __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restric
 
 cudaError_t launch_terms(const float* in, int nin, long long n, const int* ptr, const int2* term, int nout,
                          int nterm, float* out, cudaStream_t st) {
-  size_t tab = 4 * (size_t)((nout + 2) & ~1) + 8 * (size_t)nterm;
-  const int staged = tab <= 64 * 1024 ? 1 : 0;
-  if (!staged) tab = 0;
+  const size_t tab_full = 4 * (size_t)((nout + 4) & ~3) + 8 * (size_t)((nterm + 1) & ~1);
+  const int staged = tab_full <= 32 * 1024 ? 1 : 0;
+  const size_t tab = staged ? tab_full : 0;
+  // items per group: two stages, four CTAs per SM within ~55 KB of shared memory each,
+  // else two within ~110 KB
+  auto bytes = [&](int te) { return tab + 2 * (size_t)te * nin * 4; };
   int te = 32;
-  while (te > 1 && tab + (size_t)te * nin * 4 > 100 * 1024) te >>= 1;
-  const size_t sm = tab + (size_t)te * nin * 4;
+  while (te > 4 && bytes(te) > 55 * 1024) te >>= 1;
+  while (te > 1 && bytes(te) > 110 * 1024) te >>= 1;
+  const int bulk = (((uintptr_t)in & 15) == 0 && te % 4 == 0) ? 1 : 0;
+  const size_t sm = bytes(te);
   cudaError_t err = cudaFuncSetAttribute(apply_terms_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (err != cudaSuccess) return err;
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const long long groups = (n + te - 1) / te;
-  const int grid = (int)(groups < 148 * 2 ? groups : 148 * 2);
-  apply_terms_kernel<<<grid, 256, sm, st>>>(in, nin, n, ptr, term, nout, nterm, staged, te, out);
+  const int grid = (int)(groups < 4LL * nsm ? groups : 4LL * nsm);
+  apply_terms_kernel<<<grid, 256, sm, st>>>(in, nin, n, ptr, term, nout, nterm, staged, te, bulk, out);
   return cudaGetLastError();
 }
 

@@ -41,28 +41,28 @@
 
 namespace {
 
-constexpr int kXS = 3;              // x tile stages (128 edges x 64 K, bf16, 16 KB)
+constexpr int kMaxXS = 8;           // x tile stages (128 edges x 64 K, bf16, 16 KB): 3..8 per launch
 constexpr int kWS = 3;              // weight tile stages (<= 256 rows x 64 K, bf16, 32 KB)
 constexpr int kXBytes = 128 * 128;
 constexpr int kWBytes = 256 * 128;
 constexpr int kFThreads = 10 * 32;  // warp 0 bulk copies, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kEpiBar = 1;     // named barrier of the 256 epilogue threads
-constexpr int kDGroup = 6144;       // floats of dbuf per epilogue group (24 KB)
 
 struct FusedCtl {
-  uint64_t x_full[kXS], x_empty[kXS], w_full[kWS], w_empty[kWS];
+  uint64_t x_full[kMaxXS], x_empty[kMaxXS], w_full[kWS], w_empty[kWS];
   uint64_t acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
 };
 
 // Epilogue shared memory (after the operand stages).
+// The epilogue's work buffer dbuf (sized per launch, after EpiSmem) holds, in turn: the
+// partial logits of group 0's warps and their SiLU(y0) staging tiles (|m| = 0 passes),
+// the rows m = 0 of every D^l (y0 step), and per group the Wigner rows of its passes.
 struct EpiSmem {
-  float dbuf[2 * kDGroup];        // per group: Wigner rows of its passes; all: m = 0 rows, partial logits
   float pw[128 * 16];             // logits a[e][h], then softmax numerators p[e][h]
   float segS[128 * 16];           // softmax denominator of each tile segment and head
   float segM[2 * 16];             // softmax maximum of the two partial (slot) segments
-  uint16_t tst[4][32 * 32];       // per logits warp: SiLU(y0) of 32 edges x 32 channels, bf16
   int dst[128];                   // destination atom of each edge of the tile
   int seg_d[129], seg_b[129], seg_slot[129];
   int wcnt[4];
@@ -120,7 +120,7 @@ __device__ __forceinline__ void flush(float* tg, int C, float2* acc) {
 // segment's record).  The thread's stash row holds its channel's 128 edges
 // contiguously (bf16), read 32 edges at a time with the next 32 in flight.
 template <int NL>
-__device__ __noinline__ void y0_degree(const EpiArgs A, const EpiSmem* es, int t, int l, int c, int hh,
+__device__ __noinline__ void y0_degree(const EpiArgs A, const EpiSmem* es, const float* m0r, int t, int l, int c, int hh,
                                        int nvalid, int DZ, int offz, const uint4* st_row) {
   float2 acc[(NL + 1) / 2];
 #pragma unroll
@@ -146,7 +146,7 @@ __device__ __noinline__ void y0_degree(const EpiArgs A, const EpiSmem* es, int t
       if (j8 + 8 <= nb && j8 + 8 <= nvalid) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          axpy_row<NL>(acc, es->dbuf + (j8 + i) * DZ + offz, es->pw[(j8 + i) * 16 + hh] * v[i]);
+          axpy_row<NL>(acc, m0r + (j8 + i) * DZ + offz, es->pw[(j8 + i) * 16 + hh] * v[i]);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -157,7 +157,7 @@ __device__ __noinline__ void y0_degree(const EpiArgs A, const EpiSmem* es, int t
             ++k;
             nb = es->seg_b[k + 1];
           }
-          axpy_row<NL>(acc, es->dbuf + e * DZ + offz, es->pw[e * 16 + hh] * v[i]);
+          axpy_row<NL>(acc, m0r + e * DZ + offz, es->pw[e * 16 + hh] * v[i]);
         }
       }
     }
@@ -346,14 +346,16 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
   const uint32_t X_u32 = base_u32;
-  const uint32_t W_u32 = base_u32 + kXS * kXBytes;
-  EpiSmem* es = reinterpret_cast<EpiSmem*>(base + kXS * kXBytes + kWS * kWBytes);
-  FusedCtl* ctl = reinterpret_cast<FusedCtl*>(reinterpret_cast<uint8_t*>(es) + ((sizeof(EpiSmem) + 15) & ~15));
+  const int nxs = P.f_nxs;   // x stages of this launch
+  const uint32_t W_u32 = base_u32 + nxs * kXBytes;
+  EpiSmem* es = reinterpret_cast<EpiSmem*>(base + nxs * kXBytes + kWS * kWBytes);
+  float* dbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(es) + ((sizeof(EpiSmem) + 15) & ~15));
+  FusedCtl* ctl = reinterpret_cast<FusedCtl*>(dbuf + 2 * P.f_dgroup);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &ctl->abort;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kXS; ++i) {
+    for (int i = 0; i < nxs; ++i) {
       tc::mbar_init(tc::smem_u32(&ctl->x_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->x_empty[i]), 1);
     }
@@ -396,8 +398,8 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
             tc::bulk_g2s(W_u32 + sw * kWBytes, P.wprep + ps.boff + (long long)kb * bytes, bytes,
                          tc::smem_u32(&ctl->w_full[sw]));
             for (int h = 0; h < nx; ++h, ++ix) {
-              const int sx = ix % kXS;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_empty[sx]), ((ix / kXS) & 1) ^ 1, P.status, abort, 64)) break;
+              const int sx = ix % nxs;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_empty[sx]), ((ix / nxs) & 1) ^ 1, P.status, abort, 64)) break;
               const int id = ps.block == 0 ? kb : P.xbase[ps.block] + 2 * kb + h;
               tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->x_full[sx]), (uint32_t)kXBytes);
               tc::bulk_g2s(X_u32 + sx * kXBytes, xt + (long long)id * kXBytes, (uint32_t)kXBytes,
@@ -413,10 +415,10 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         while (!tc::mbar_try_wait(bar, (k / kWS) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
         }
       }
-      for (uint32_t k = (ix > (uint32_t)kXS ? ix - kXS : 0); k < ix; ++k) {
-        const uint32_t bar = tc::smem_u32(&ctl->x_full[k % kXS]);
+      for (uint32_t k = (ix > (uint32_t)nxs ? ix - nxs : 0); k < ix; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->x_full[k % nxs]);
         const uint64_t t0 = tc::globaltimer();
-        while (!tc::mbar_try_wait(bar, (k / kXS) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        while (!tc::mbar_try_wait(bar, (k / nxs) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
         }
       }
     }
@@ -435,10 +437,10 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           if (ps.block > 0) {
             // y+ += W1 x+ - W2 x- (columns 0-127); y- += W2 x+ + W1 x- (columns 128-255)
             for (int kb = 0; kb < ps.nk; ++kb, ++iw, ix += 2) {
-              const int sw = iw % kWS, sp = ix % kXS, sm = (ix + 1) % kXS;
+              const int sw = iw % kWS, sp = ix % nxs, sm = (ix + 1) % nxs;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / kWS) & 1, P.status, abort)) break;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sp]), (ix / kXS) & 1, P.status, abort)) break;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sm]), ((ix + 1) / kXS) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sp]), (ix / nxs) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sm]), ((ix + 1) / nxs) & 1, P.status, abort)) break;
               tc::tc_fence_after();
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
@@ -459,9 +461,9 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           } else {
             const int nrb = ps.n / 128;   // one or two degrees of y0
             for (int kb = 0; kb < ps.nk; ++kb, ++iw, ++ix) {
-              const int sw = iw % kWS, sx = ix % kXS;
+              const int sw = iw % kWS, sx = ix % nxs;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / kWS) & 1, P.status, abort)) break;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sx]), (ix / kXS) & 1, P.status, abort)) break;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sx]), (ix / nxs) & 1, P.status, abort)) break;
               tc::tc_fence_after();
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
     const int C = P.C, H = P.H, L = P.L, L2 = P.L2, hh = c / (C / H);
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     __nv_bfloat16* stash = P.stash + (size_t)blockIdx.x * L * 128 * C;
-    float* dg = es->dbuf + g * kDGroup;                    // this group's Wigner rows
+    float* dg = dbuf + g * P.f_dgroup;                     // this group's Wigner rows
     const EpiArgs EA{P.slots, P.acc_g, P.C, P.L2, P.rec_floats};
     int DZ = 0;
     for (int l = 0; l < L; ++l) DZ += pad4(2 * l + 1);
@@ -541,13 +543,13 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         }
       }
       // ---- |m| = 0 passes: group 0 SiLU(y0) into the logits, group 1 y0 into the stash ----
-      float* Lp = es->dbuf;   // [4][128][H] partial logits of group 0's warps
+      float* Lp = dbuf;   // [4][128][H] partial logits of group 0's warps, then their staging tiles
       if (g == 0) {
         for (int i = lane; i < 128 * H; i += 32) Lp[q * 128 * H + i] = 0.f;
         __syncwarp();
       }
       int p = 0;
-      uint16_t* T = es->tst[q];
+      uint16_t* T = reinterpret_cast<uint16_t*>(dbuf + 4 * 128 * H) + q * 32 * 32;
       const uint32_t T_u32 = tc::smem_u32(T);
       for (; p < P.npass && P.pass[p].block == 0; ++p, ++ip) {
         const TcPass& ps = P.pass[p];
@@ -576,28 +578,11 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         }
       }
       epi_bar();
-      {
-        const int ns = es->nseg;
-        for (int pr = et; pr < ns * H; pr += 256) {
-          const int k = pr / H, h = pr - k * H;
-          const int b = es->seg_b[k], en = es->seg_b[k + 1];
-          float mx = -INFINITY;
-          for (int e = b; e < en; ++e) mx = fmaxf(mx, es->pw[e * 16 + h]);
-          float sum = 0.f;
-          for (int e = b; e < en; ++e) {
-            const float x = __expf(es->pw[e * 16 + h] - mx);
-            es->pw[e * 16 + h] = x;
-            sum += x;
-          }
-          es->segS[k * 16 + h] = sum;
-          const int slot = es->seg_slot[k];
-          if (slot >= 0) es->segM[slot * 16 + h] = mx;
-        }
-      }
-      // ---- rows m = 0 of every D^l for the tile (one edge per thread of group 0) ----
+      // ---- rows m = 0 of every D^l for the tile (one edge per thread of group 0), fetched
+      // asynchronously while the softmax statistics are formed (Lp is no longer needed) ----
       if (et < nvalid && et < 128) {
         const float* wr = P.wig + (size_t)(e0 + et) * P.wfl;
-        const uint32_t dz = tc::smem_u32(es->dbuf + et * DZ);
+        const uint32_t dz = tc::smem_u32(dbuf + et * DZ);
         int off = 0;
         for (int l = 0; l < L; ++l) {
           const int ml = l < P.mmax ? l : P.mmax, dl = 2 * l + 1;
@@ -605,8 +590,33 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           for (int m = 0; m < dl; ++m) tc::cp_async4(dz + 4 * (off + m), row + m);
           off += pad4(dl);
         }
-        tc::cp_async_wait_all();
       }
+      // ---- softmax statistics per (segment, head): one warp per pair, lanes over edges ----
+      {
+        const int ns = es->nseg, ew = et >> 5;
+        for (int pr = ew; pr < ns * H; pr += 8) {
+          const int k = pr / H, h = pr - k * H;
+          const int b = es->seg_b[k], en = es->seg_b[k + 1];
+          float mx = -INFINITY;
+          for (int e = b + lane; e < en; e += 32) mx = fmaxf(mx, es->pw[e * 16 + h]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          float sum = 0.f;
+          for (int e = b + lane; e < en; e += 32) {
+            const float x = __expf(es->pw[e * 16 + h] - mx);
+            es->pw[e * 16 + h] = x;
+            sum += x;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          if (lane == 0) {
+            es->segS[k * 16 + h] = sum;
+            const int slot = es->seg_slot[k];
+            if (slot >= 0) es->segM[slot * 16 + h] = mx;
+          }
+        }
+      }
+      if (et < nvalid && et < 128) tc::cp_async_wait_all();
       epi_bar();
       // ---- y0 from the stash, degrees of this group: first contribution of each record ----
       {
@@ -615,13 +625,13 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           if (own_deg(P, g, l)) {
             const uint4* st_row = reinterpret_cast<const uint4*>(stash + ((size_t)l * C + c) * 128);
             switch (l) {
-              case 0: y0_degree<1>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 1: y0_degree<3>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 2: y0_degree<5>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 3: y0_degree<7>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 4: y0_degree<9>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 5: y0_degree<11>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              default: y0_degree<13>(EA, es, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 0: y0_degree<1>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 1: y0_degree<3>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 2: y0_degree<5>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 3: y0_degree<7>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 4: y0_degree<9>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              case 5: y0_degree<11>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+              default: y0_degree<13>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
             }
           }
           offz += pad4(2 * l + 1);
@@ -633,7 +643,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       // (one or two buffers); the next own pass's rows are fetched asynchronously while
       // the current pass is summed when both fit.
       const int pass_floats = 128 * 2 * pad4(2 * L - 1);
-      const bool dbl = 2 * pass_floats <= kDGroup;
+      const bool dbl = 2 * pass_floats <= P.f_dgroup;
       int pown = p;
       while (pown < P.npass && !own_deg(P, g, pass_l(P, pown))) ++pown;
       int half = 0;
@@ -767,12 +777,40 @@ __global__ void edge_dst_kernel(const int32_t* __restrict__ row_ptr, int n_atoms
   for (int e = row_ptr[d] + lane; e < row_ptr[d + 1]; e += 32) dst[e] = d;
 }
 
-size_t fused_smem_total() {
-  return kXS * kXBytes + kWS * kWBytes + ((sizeof(EpiSmem) + 15) & ~(size_t)15) + sizeof(FusedCtl) + 1024;
+// Shared memory of one launch: x stages, weight stages, EpiSmem, dbuf, control block
+// (+ 1 KB to align the operand stages to 1024 bytes).
+size_t fused_smem_bytes(int nxs, int dgroup) {
+  return (size_t)nxs * kXBytes + kWS * kWBytes + ((sizeof(EpiSmem) + 15) & ~(size_t)15) +
+         sizeof(float) * 2 * (size_t)dgroup + sizeof(FusedCtl) + 1024;
+}
+
+#ifndef EGNN_FUSED_DOUBLE_ROWS
+#define EGNN_FUSED_DOUBLE_ROWS 0
+#endif
+
+// dbuf size and x stage count: dbuf holds the largest of its three uses (partial logits
+// and staging tiles, the m = 0 rows of a tile, each group's pass rows, single- or
+// double-buffered); the x stages take what shared memory is left, up to kMaxXS.
+bool fused_layout(const TcParams& P, int& nxs, int& dgroup) {
+  int DZ = 0;   // floats of one edge's m = 0 rows, each row padded to four floats
+  for (int l = 0; l < P.L; ++l) DZ += ((2 * l + 1) + 3) & ~3;
+  const int need_lp = 4 * 128 * P.H + 4 * 32 * 32 / 2;       // partial logits + bf16 tiles
+  const int need_m0 = 128 * DZ;
+  const int pass_floats = 128 * 2 * (((2 * P.L - 1) + 3) & ~3);
+  const int need_rows = (EGNN_FUSED_DOUBLE_ROWS ? 4 : 2) * pass_floats;
+  int dbuf = need_lp > need_m0 ? need_lp : need_m0;
+  if (need_rows > dbuf) dbuf = need_rows;
+  dbuf = (dbuf + 7) & ~7;
+  dgroup = dbuf / 2;
+  int dev = 0, optin = 232448;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  for (nxs = kMaxXS; nxs >= 3; --nxs)
+    if (fused_smem_bytes(nxs, dgroup) <= (size_t)optin) return true;
+  return false;
 }
 
 cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*) {
-  const size_t sm = fused_smem_total();
+  const size_t sm = fused_smem_bytes(Ps.f_nxs, Ps.f_dgroup);
   cudaError_t err = cudaFuncSetAttribute(layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (err != cudaSuccess) return err;
   layer_fused_kernel<<<grid, kFThreads, sm, st>>>(Ps);
@@ -781,11 +819,11 @@ cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*)
 
 }  // namespace
 
-size_t layer_fused_smem_bytes(int, int) { return fused_smem_total(); }
-
 // Destination of every edge, weight prep, then per range of edge tiles: gates and rotation
 // -> fused SO(2) layer; then the destinations that cross tile boundaries or have none.
-cudaError_t launch_layer_fused(const TcParams& P, const TcWeights& W, cudaStream_t st) {
+cudaError_t launch_layer_fused(const TcParams& P0, const TcWeights& W, cudaStream_t st) {
+  TcParams P = P0;
+  if (!fused_layout(P, P.f_nxs, P.f_dgroup)) return cudaErrorInvalidValue;
   if (P.n_edges > 0) edge_dst_kernel<<<(P.n_atoms * 32 + 255) / 256, 256, 0, st>>>(P.row_ptr, P.n_atoms, P.edge_dst);
   cudaError_t err = launch_tc_pipeline(P, W, st, fused_consumer, nullptr, true);
   if (err != cudaSuccess) return err;

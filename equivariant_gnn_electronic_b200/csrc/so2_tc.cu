@@ -300,27 +300,39 @@ __host__ __device__ inline HeadTabWords head_tab_words(int n_lab, int n_entries,
 // h[L, M, k] = sum_m D^L[m, M] s[L, m, k] (one thread per label), and each block entry
 // is the sum of the Clebsch-Gordan images of its shell pair's labels (one thread per
 // entry).  The rotation commutes with U^L because U^L mixes channels only.
-// Per group of te edges (persistent CTAs): records and Wigner rows staged in shared
-// memory; every label from its precomputed list of (Wigner offset, record offset) pairs;
-// every block entry from its precomputed list of (label, Clebsch-Gordan coefficient)
-// terms (both built on the host from the orbital template and the pass layout).
+// Per group of te edges (persistent CTAs): the group's records and Wigner rows arrive by
+// 1-D bulk copies into one of two shared-memory stages, one group ahead (a ragged last
+// group whose Wigner bytes are not a multiple of 16 is loaded by all threads); every
+// label from its precomputed list of (Wigner offset, record offset) pairs; every block
+// entry from its precomputed list of (label, Clebsch-Gordan coefficient) terms (both
+// built on the host from the orbital template and the pass layout).  Work items are
+// (edge, label) and (edge, entry) pairs, so the block stores are contiguous.
 __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__ TcParams P,
                                                          const __grid_constant__ HeadLabelTabs Tb,
-                                                         float* __restrict__ blocks, int te, int staged) {
-  extern __shared__ float hsm[];
-  const int nrec = P.y_row_bytes / 4, wfl4 = (P.wfl + 3) & ~3;
+                                                         float* __restrict__ blocks, int te, int staged, int bulk) {
+  extern __shared__ __align__(16) float hsm[];
+  __shared__ uint64_t full[2];
+  __shared__ int abort_flag;
+  const int nrec = P.y_row_bytes / 4, wfl = P.wfl;
   const int nlab = Tb.n_lab, nb = Tb.n_orb * Tb.n_orb, nterm = staged ? Tb.n_term : 0;
   // tables staged once per CTA when small (label terms [nlab][11], entry term pointers,
-  // terms), each region starting on a 16-byte boundary (the terms are read as int2, the
-  // records behind them as float4); otherwise read through the read-only cache
+  // terms), each region starting on a 16-byte boundary (the terms are read as int2);
+  // otherwise read through the read-only cache
   const HeadTabWords tw = head_tab_words(nlab, nb, Tb.n_term, staged != 0);
   int* s_lab = reinterpret_cast<int*>(hsm);
   int* s_tptr = s_lab + tw.lab;
   int2* s_term = reinterpret_cast<int2*>(s_tptr + tw.tptr);
-  float* Rs = reinterpret_cast<float*>(s_tptr + tw.tptr + tw.term);   // [te][nrec]
-  float* Ds = Rs + te * nrec;                              // [te][wfl4]
-  float* Ls = Ds + te * wfl4;                              // [te][nlab]
+  // two stages of [te][nrec] records + [te][wfl] Wigner rows, then the labels [te][nlab]
+  float* stage0 = reinterpret_cast<float*>(s_tptr + tw.tptr + tw.term);
+  const int stage_floats = te * (nrec + wfl);
+  float* Ls = stage0 + 2 * stage_floats;
   const int tid = threadIdx.x, nt = blockDim.x;
+  if (tid == 0) {
+    tc::mbar_init(tc::smem_u32(&full[0]), 1);
+    tc::mbar_init(tc::smem_u32(&full[1]), 1);
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
   if (staged) {
     for (int i = tid; i < nlab * 11; i += nt) s_lab[i] = Tb.lab[i];
     for (int i = tid; i <= nb; i += nt) s_tptr[i] = Tb.term_ptr[i];
@@ -330,42 +342,95 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
     s_tptr = const_cast<int*>(Tb.term_ptr);
     s_term = const_cast<int2*>(Tb.term);
   }
+  __syncthreads();
   const long long ngroups = (P.n_edges + te - 1) / te;
-  for (long long gi = blockIdx.x; gi < ngroups; gi += gridDim.x) {
+  // a group's records and Wigner rows are each contiguous in global memory: two 1-D
+  // bulk copies on one barrier when the Wigner byte count is a multiple of 16
+  auto by_copy = [&](long long gi) {
+    return bulk && ((min((long long)te, P.n_edges - gi * te) * wfl) & 3) == 0;
+  };
+  auto issue = [&](long long gi, int st) {   // thread 0 only
     const long long e0 = gi * te;
     const int ne = (int)min((long long)te, P.n_edges - e0);
-    __syncthreads();
-    {
+    const uint32_t rb = (uint32_t)ne * P.y_row_bytes, wb = (uint32_t)ne * wfl * 4;
+    const uint32_t bar = tc::smem_u32(&full[st]);
+    float* S = stage0 + st * stage_floats;
+    tc::mbar_arrive_expect_tx(bar, rb + wb);
+    tc::bulk_g2s(tc::smem_u32(S), P.Y + e0 * (long long)P.y_row_bytes, rb, bar);
+    tc::bulk_g2s(tc::smem_u32(S + te * nrec), P.wig + e0 * wfl, wb, bar);
+  };
+  uint32_t phase[2] = {0u, 0u};
+  bool pend[2] = {false, false};   // thread 0: a copy into the stage is in flight
+  int it = 0;
+  if (tid == 0 && blockIdx.x < ngroups && by_copy(blockIdx.x)) {
+    issue(blockIdx.x, 0);
+    pend[0] = true;
+  }
+  for (long long gi = blockIdx.x; gi < ngroups; gi += gridDim.x, ++it) {
+    const int st = it & 1;
+    const long long e0 = gi * te;
+    const int ne = (int)min((long long)te, P.n_edges - e0);
+    const long long gn = gi + gridDim.x;
+    if (tid == 0 && gn < ngroups && by_copy(gn)) {
+      issue(gn, st ^ 1);
+      pend[st ^ 1] = true;
+    }
+    float* Rs = stage0 + st * stage_floats;
+    float* Ds = Rs + te * nrec;
+    if (by_copy(gi)) {
+      const bool ok = tc::mbar_wait(tc::smem_u32(&full[st]), phase[st], P.status, &abort_flag, 0);
+      if (!__syncthreads_and(ok)) break;
+      phase[st] ^= 1u;
+      pend[st] = false;
+    } else {
       const float4* rsrc = reinterpret_cast<const float4*>(P.Y + e0 * (long long)P.y_row_bytes);
       float4* rdst = reinterpret_cast<float4*>(Rs);
       for (int i = tid; i < ne * nrec / 4; i += nt) rdst[i] = rsrc[i];
-      const float* wsrc = P.wig + e0 * P.wfl;
-      for (int e = 0; e < ne; ++e)
-        for (int i = tid; i < P.wfl; i += nt) Ds[e * wfl4 + i] = wsrc[(long long)e * P.wfl + i];
+      for (int i = tid; i < ne * wfl; i += nt) Ds[i] = P.wig[e0 * wfl + i];
+      __syncthreads();
     }
-    __syncthreads();
-    for (int q = tid; q < nlab; q += nt) {
-      const int* lt = s_lab + q * 11;
-      const int cnt = lt[0];
-      for (int e = 0; e < ne; ++e) {
-        const float* De = Ds + e * wfl4;
+    // labels, one (edge, label) per work item: Ls[e][q] is item e * nlab + q
+    {
+      int e = tid / nlab, q = tid - e * nlab;
+      for (int w = tid; w < ne * nlab; w += nt) {
+        const int* lt = s_lab + q * 11;
+        const int cnt = lt[0];
+        const float* De = Ds + e * wfl;
         const float* Re = Rs + e * nrec;
         float h = 0.f;
         for (int j = 0; j < cnt; ++j) h = fmaf(De[lt[1 + j]], Re[lt[6 + j]], h);
-        Ls[e * nlab + q] = h;
+        Ls[w] = h;
+        q += nt;
+        while (q >= nlab) { q -= nlab; ++e; }
       }
     }
     __syncthreads();
-    for (int q = tid; q < nb; q += nt) {
-      const int t0 = s_tptr[q], t1 = s_tptr[q + 1];
-      for (int e = 0; e < ne; ++e) {
+    // block entries, one (edge, entry) per work item: consecutive items are consecutive
+    // entries of the group's output, so the stores are contiguous
+    {
+      int e = tid / nb, q = tid - e * nb;
+      float* out = blocks + e0 * nb;
+      for (int w = tid; w < ne * nb; w += nt) {
         const float* Le = Ls + e * nlab;
+        const int t1 = s_tptr[q + 1];
         float v = 0.f;
-        for (int t = t0; t < t1; ++t) {
+        for (int t = s_tptr[q]; t < t1; ++t) {
           const int2 tm = s_term[t];
           v = fmaf(__int_as_float(tm.y), Le[tm.x], v);
         }
-        blocks[(e0 + e) * nb + q] = v;
+        out[w] = v;
+        q += nt;
+        while (q >= nb) { q -= nb; ++e; }
+      }
+    }
+    __syncthreads();   // stage st and Ls are free for the next iteration
+  }
+  // a copy still in flight (only after a wait ran out) must land before the CTA exits
+  if (tid == 0) {
+    for (int st = 0; st < 2; ++st) {
+      if (!pend[st]) continue;
+      const uint64_t t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(tc::smem_u32(&full[st]), phase[st]) && tc::globaltimer() - t0 < 2000000000ull) {
       }
     }
   }
@@ -648,6 +713,23 @@ __global__ void __launch_bounds__(kGRThreads, 1) gate_rotate_kernel(const __grid
         for (int r = rw; r < 128; r += kGRRot) {
           const long long e = (long long)t * 128 + r;
           const bool valid = e < E;
+          {
+            // L2 hint for the node rows and Wigner coefficients of this warp's edge two
+            // iterations ahead, so that the loads below meet L2 rather than HBM
+            // (source rows: two 128-byte lines per row; the destination's rows repeat
+            // from edge to edge and stay cached)
+            const int rp = r + 2 * kGRRot;
+            if (rp < 128 && e + 2 * kGRRot < E) {
+              if (lane < 2 * dl) {
+                const long long row = (long long)ctl->node[0][rp] * (L * L) + l * l + (lane >> 1);
+                tc::prefetch_l2(P.node_in + row * 128 + (lane & 1) * 64);
+              } else if (lane < 2 * dl + 3) {
+                const int k = lane - 2 * dl, last = nr * dl - 1;
+                const int off = 32 * k < last ? 32 * k : last;
+                tc::prefetch_l2(P.wig + (e + 2 * kGRRot) * (long long)P.wfl + wo + off);
+              }
+            }
+          }
           const __nv_bfloat16* zn =
               P.node_in + ((long long)ctl->node[side][r] * (L * L) + l * l) * 128 + (lane & 15) * 8;
           const float* De = P.wig + (valid ? e : 0) * (long long)P.wfl + wo;
@@ -1054,19 +1136,23 @@ cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTabl
     const int nb = LT.n_orb * LT.n_orb;
     const HeadTabWords tw = head_tab_words(LT.n_lab, nb, LT.n_term, true);
     size_t tab = 4 * ((size_t)tw.lab + tw.tptr + tw.term);
-    const int staged = tab <= 64 * 1024 ? 1 : 0;
+    const int staged = tab <= 24 * 1024 ? 1 : 0;
     if (!staged) tab = 0;
+    // two stages of records and Wigner rows, then the group's labels
     auto bytes = [&](int t) {
-      return tab + sizeof(float) * (size_t)t * (size_t)(P.y_row_bytes / 4 + ((P.wfl + 3) & ~3) + T.n_lab);
+      return tab + sizeof(float) * (size_t)t * (size_t)(2 * (P.y_row_bytes / 4 + P.wfl) + T.n_lab);
     };
-    int te = 32;   // edges per group: two CTAs per SM within ~110 KB of shared memory each
+    int te = 32;   // edges per group: three CTAs per SM within ~72 KB of shared memory each,
+    while (te > 4 && bytes(te) > 72 * 1024) te >>= 1;   // else two within ~110 KB
     while (te > 1 && bytes(te) > 110 * 1024) te >>= 1;
     if (bytes(te) > 220 * 1024) return cudaErrorInvalidValue;
+    // bulk copies need 16-byte aligned sources and groups that start on 16-byte boundaries
+    const int bulk = (((uintptr_t)P.wig | (uintptr_t)P.Y) & 15) == 0 && te % 4 == 0 && P.y_row_bytes % 16 == 0;
     err = cudaFuncSetAttribute(head_label_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes(te));
     if (err != cudaSuccess) return err;
     const long long groups = (P.n_edges + te - 1) / te;
-    const int grid = (int)(groups < 4LL * P.grid ? groups : 4LL * P.grid);
-    head_label_kernel<<<grid, 256, bytes(te), st>>>(P, LT, blocks, te, staged);
+    const int grid = (int)(groups < 3LL * P.grid ? groups : 3LL * P.grid);
+    head_label_kernel<<<grid, 256, bytes(te), st>>>(P, LT, blocks, te, staged, bulk);
     return cudaGetLastError();
   }
   int u_total = 0;

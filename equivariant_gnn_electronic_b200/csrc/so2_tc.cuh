@@ -68,6 +68,7 @@ struct TcParams {
   float* slots;
   int rec_floats;
   int own_b;                     // bit l set: the fused layer's second epilogue group owns degree l
+  int f_nxs, f_dgroup;           // fused layer: x stages, floats of its work buffer per epilogue group
   int npass;
   TcPass pass[32];
   int woff[8];
@@ -118,7 +119,6 @@ using TcConsumer = cudaError_t (*)(const TcParams& Ps, int grid, cudaStream_t st
 cudaError_t launch_tc_pipeline(const TcParams& P, const TcWeights& W, cudaStream_t st, TcConsumer consumer,
                                void* ctx, bool profiled);
 cudaError_t launch_layer_fused(const TcParams& P, const TcWeights& W, cudaStream_t st);
-size_t layer_fused_smem_bytes(int lmax, int heads);
 cudaError_t launch_head_tc(const TcParams& P, const TcWeights& W, const HeadTables& T, HeadUPtrs U,
                            const HeadLabelTabs& LT, float* blocks, cudaStream_t st);
 size_t head_tc_smem_bytes(const TcParams& P, int n_lab, int te);

@@ -42,14 +42,14 @@
 namespace {
 
 constexpr int kMaxXS = 8;           // x tile stages (128 edges x 64 K, bf16, 16 KB): 3..8 per launch
-constexpr int kWS = 3;              // weight tile stages (<= 256 rows x 64 K, bf16, 32 KB)
+constexpr int kMaxWS = 3;           // weight tile stages (<= 256 rows x 64 K, bf16, 32 KB): 2..3 per launch
 constexpr int kXBytes = 128 * 128;
 constexpr int kWBytes = 256 * 128;
 constexpr int kFThreads = 10 * 32;  // warp 0 bulk copies, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kEpiBar = 1;     // named barrier of the 256 epilogue threads
 
 struct FusedCtl {
-  uint64_t x_full[kMaxXS], x_empty[kMaxXS], w_full[kWS], w_empty[kWS];
+  uint64_t x_full[kMaxXS], x_empty[kMaxXS], w_full[kMaxWS], w_empty[kMaxWS];
   uint64_t acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
@@ -346,11 +346,14 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
   const uint32_t X_u32 = base_u32;
-  const int nxs = P.f_nxs;   // x stages of this launch
+  const int nxs = P.f_nxs, nws = P.f_nws;   // x and weight stages of this launch
   const uint32_t W_u32 = base_u32 + nxs * kXBytes;
-  EpiSmem* es = reinterpret_cast<EpiSmem*>(base + nxs * kXBytes + kWS * kWBytes);
+  EpiSmem* es = reinterpret_cast<EpiSmem*>(base + nxs * kXBytes + nws * kWBytes);
   float* dbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(es) + ((sizeof(EpiSmem) + 15) & ~15));
-  FusedCtl* ctl = reinterpret_cast<FusedCtl*>(dbuf + 2 * P.f_dgroup);
+  int DZ = 0;   // floats of one edge's m = 0 rows of every D^l, each row padded to four floats
+  for (int l = 0; l < P.L; ++l) DZ += pad4(2 * l + 1);
+  float* m0r = dbuf + 2 * P.f_dgroup;   // [128][DZ]: the tile's m = 0 rows, kept for the whole tile
+  FusedCtl* ctl = reinterpret_cast<FusedCtl*>(m0r + 128 * DZ);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &ctl->abort;
 
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       tc::mbar_init(tc::smem_u32(&ctl->x_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->x_empty[i]), 1);
     }
-    for (int i = 0; i < kWS; ++i) {
+    for (int i = 0; i < nws; ++i) {
       tc::mbar_init(tc::smem_u32(&ctl->w_full[i]), 1);
       tc::mbar_init(tc::smem_u32(&ctl->w_empty[i]), 1);
     }
@@ -392,8 +395,8 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           const uint32_t bytes = (uint32_t)ps.n * 128u;
           const int nx = ps.block > 0 ? 2 : 1;
           for (int kb = 0; kb < ps.nk && !*abort; ++kb, ++iw) {
-            const int sw = iw % kWS;
-            if (!tc::mbar_wait(tc::smem_u32(&ctl->w_empty[sw]), ((iw / kWS) & 1) ^ 1, P.status, abort, 64)) break;
+            const int sw = iw % nws;
+            if (!tc::mbar_wait(tc::smem_u32(&ctl->w_empty[sw]), ((iw / nws) & 1) ^ 1, P.status, abort, 64)) break;
             tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->w_full[sw]), bytes);
             tc::bulk_g2s(W_u32 + sw * kWBytes, P.wprep + ps.boff + (long long)kb * bytes, bytes,
                          tc::smem_u32(&ctl->w_full[sw]));
@@ -409,10 +412,10 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         }
       }
       // the newest phase of every stage must have landed before the CTA exits
-      for (uint32_t k = (iw > (uint32_t)kWS ? iw - kWS : 0); k < iw; ++k) {
-        const uint32_t bar = tc::smem_u32(&ctl->w_full[k % kWS]);
+      for (uint32_t k = (iw > (uint32_t)nws ? iw - nws : 0); k < iw; ++k) {
+        const uint32_t bar = tc::smem_u32(&ctl->w_full[k % nws]);
         const uint64_t t0 = tc::globaltimer();
-        while (!tc::mbar_try_wait(bar, (k / kWS) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
+        while (!tc::mbar_try_wait(bar, (k / nws) & 1) && tc::globaltimer() - t0 < 2000000000ull) {
         }
       }
       for (uint32_t k = (ix > (uint32_t)nxs ? ix - nxs : 0); k < ix; ++k) {
@@ -437,8 +440,8 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           if (ps.block > 0) {
             // y+ += W1 x+ - W2 x- (columns 0-127); y- += W2 x+ + W1 x- (columns 128-255)
             for (int kb = 0; kb < ps.nk; ++kb, ++iw, ix += 2) {
-              const int sw = iw % kWS, sp = ix % nxs, sm = (ix + 1) % nxs;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / kWS) & 1, P.status, abort)) break;
+              const int sw = iw % nws, sp = ix % nxs, sm = (ix + 1) % nxs;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / nws) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sp]), (ix / nxs) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sm]), ((ix + 1) / nxs) & 1, P.status, abort)) break;
               tc::tc_fence_after();
@@ -461,8 +464,8 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           } else {
             const int nrb = ps.n / 128;   // one or two degrees of y0
             for (int kb = 0; kb < ps.nk; ++kb, ++iw, ++ix) {
-              const int sw = iw % kWS, sx = ix % nxs;
-              if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / kWS) & 1, P.status, abort)) break;
+              const int sw = iw % nws, sx = ix % nxs;
+              if (!tc::mbar_wait(tc::smem_u32(&ctl->w_full[sw]), (iw / nws) & 1, P.status, abort)) break;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->x_full[sx]), (ix / nxs) & 1, P.status, abort)) break;
               tc::tc_fence_after();
 #pragma unroll
@@ -504,8 +507,6 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
     __nv_bfloat16* stash = P.stash + (size_t)blockIdx.x * L * 128 * C;
     float* dg = dbuf + g * P.f_dgroup;                     // this group's Wigner rows
     const EpiArgs EA{P.slots, P.acc_g, P.C, P.L2, P.rec_floats};
-    int DZ = 0;
-    for (int l = 0; l < L; ++l) DZ += pad4(2 * l + 1);
     uint32_t ip = 0;
     bool failed = false;
     for (int t = P.t_begin + blockIdx.x; t < P.t_end && !failed; t += gridDim.x) {
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       // asynchronously while the softmax statistics are formed (Lp is no longer needed) ----
       if (et < nvalid && et < 128) {
         const float* wr = P.wig + (size_t)(e0 + et) * P.wfl;
-        const uint32_t dz = tc::smem_u32(dbuf + et * DZ);
+        const uint32_t dz = tc::smem_u32(m0r + et * DZ);
         int off = 0;
         for (int l = 0; l < L; ++l) {
           const int ml = l < P.mmax ? l : P.mmax, dl = 2 * l + 1;
@@ -618,26 +619,26 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       }
       if (et < nvalid && et < 128) tc::cp_async_wait_all();
       epi_bar();
-      // ---- y0 from the stash, degrees of this group: first contribution of each record ----
-      {
+      // ---- y0 contributions (first contribution of each record) and (+m, -m) passes ----
+      // The group's y0 step of degree l comes right before the degree's first (+m, -m)
+      // pass; the others run while the MMA works on passes the group does not own.
+      auto y0_step = [&](int l) {
         int offz = 0;
-        for (int l = 0; l < L; ++l) {
-          if (own_deg(P, g, l)) {
-            const uint4* st_row = reinterpret_cast<const uint4*>(stash + ((size_t)l * C + c) * 128);
-            switch (l) {
-              case 0: y0_degree<1>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 1: y0_degree<3>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 2: y0_degree<5>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 3: y0_degree<7>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 4: y0_degree<9>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              case 5: y0_degree<11>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-              default: y0_degree<13>(EA, es, dbuf, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-            }
-          }
-          offz += pad4(2 * l + 1);
+        for (int q2 = 0; q2 < l; ++q2) offz += pad4(2 * q2 + 1);
+        const uint4* st_row = reinterpret_cast<const uint4*>(stash + ((size_t)l * C + c) * 128);
+        switch (l) {
+          case 0: y0_degree<1>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 1: y0_degree<3>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 2: y0_degree<5>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 3: y0_degree<7>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 4: y0_degree<9>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 5: y0_degree<11>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          default: y0_degree<13>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
         }
-      }
-      epi_bar();   // dbuf (m = 0 rows) is rewritten per group below
+      };
+      unsigned y0_left = 0;
+      for (int l = 0; l < L; ++l)
+        if (own_deg(P, g, l)) y0_left |= 1u << l;
       // ---- (+m, -m) passes: each processed by the group owning its degree ----
       // The group's Wigner rows (l, +b), (l, -b) of a pass sit in dg as [e][2][pad4(2l+1)]
       // (one or two buffers); the next own pass's rows are fetched asynchronously while
@@ -654,11 +655,24 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
       group_bar(g);
       for (; p < P.npass; ++p, ++ip) {
         const int buf = ip & 1;
+        const int l = pass_l(P, p);
+        if (own_deg(P, g, l)) {
+          if ((y0_left >> l) & 1u) {
+            y0_step(l);
+            y0_left &= ~(1u << l);
+          }
+        } else if (y0_left) {
+          // the degree of the group's next own pass if still pending, else the lowest
+          const int po = next_own(P, g, p);
+          int ly = po < P.npass ? pass_l(P, po) : -1;
+          if (ly < 0 || !((y0_left >> ly) & 1u)) ly = __ffs(y0_left) - 1;
+          y0_step(ly);
+          y0_left &= ~(1u << ly);
+        }
         if (!tc::mbar_wait(tc::smem_u32(&ctl->acc_full[buf]), (ip >> 1) & 1, P.status, &no_abort, 64)) {
           failed = true;
           break;
         }
-        const int l = pass_l(P, p);
         if (own_deg(P, g, l)) {
           const int pn = next_own(P, g, p);
           float* dcur = dg + half * (dbl ? pass_floats : 0);
@@ -689,6 +703,11 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         }
       }
       if (failed) break;
+      while (y0_left) {   // degrees without (+m, -m) passes, or not yet reached
+        const int ly = __ffs(y0_left) - 1;
+        y0_step(ly);
+        y0_left &= ~(1u << ly);
+      }
       asm volatile("" ::: "memory");   // the record reads below follow this thread's adds
       // ---- finish the destinations whose edges all lie in this tile (rows of own degrees) ----
       {
@@ -779,9 +798,11 @@ __global__ void edge_dst_kernel(const int32_t* __restrict__ row_ptr, int n_atoms
 
 // Shared memory of one launch: x stages, weight stages, EpiSmem, dbuf, control block
 // (+ 1 KB to align the operand stages to 1024 bytes).
-size_t fused_smem_bytes(int nxs, int dgroup) {
-  return (size_t)nxs * kXBytes + kWS * kWBytes + ((sizeof(EpiSmem) + 15) & ~(size_t)15) +
-         sizeof(float) * 2 * (size_t)dgroup + sizeof(FusedCtl) + 1024;
+size_t fused_smem_bytes(int nxs, int nws, int dgroup, int L) {
+  int DZ = 0;
+  for (int l = 0; l < L; ++l) DZ += ((2 * l + 1) + 3) & ~3;
+  return (size_t)nxs * kXBytes + (size_t)nws * kWBytes + ((sizeof(EpiSmem) + 15) & ~(size_t)15) +
+         sizeof(float) * (2 * (size_t)dgroup + 128 * (size_t)DZ) + sizeof(FusedCtl) + 1024;
 }
 
 #ifndef EGNN_FUSED_DOUBLE_ROWS
@@ -791,26 +812,27 @@ size_t fused_smem_bytes(int nxs, int dgroup) {
 // dbuf size and x stage count: dbuf holds the largest of its three uses (partial logits
 // and staging tiles, the m = 0 rows of a tile, each group's pass rows, single- or
 // double-buffered); the x stages take what shared memory is left, up to kMaxXS.
-bool fused_layout(const TcParams& P, int& nxs, int& dgroup) {
+bool fused_layout(const TcParams& P, int& nxs, int& nws, int& dgroup) {
   int DZ = 0;   // floats of one edge's m = 0 rows, each row padded to four floats
   for (int l = 0; l < P.L; ++l) DZ += ((2 * l + 1) + 3) & ~3;
+  (void)DZ;   // the m = 0 rows have their own region after dbuf
   const int need_lp = 4 * 128 * P.H + 4 * 32 * 32 / 2;       // partial logits + bf16 tiles
-  const int need_m0 = 128 * DZ;
   const int pass_floats = 128 * 2 * (((2 * P.L - 1) + 3) & ~3);
   const int need_rows = (EGNN_FUSED_DOUBLE_ROWS ? 4 : 2) * pass_floats;
-  int dbuf = need_lp > need_m0 ? need_lp : need_m0;
-  if (need_rows > dbuf) dbuf = need_rows;
+  int dbuf = need_lp > need_rows ? need_lp : need_rows;
   dbuf = (dbuf + 7) & ~7;
   dgroup = dbuf / 2;
   int dev = 0, optin = 232448;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  for (nxs = kMaxXS; nxs >= 3; --nxs)
-    if (fused_smem_bytes(nxs, dgroup) <= (size_t)optin) return true;
+  // three weight stages with at least four x stages, else two weight stages
+  for (nws = kMaxWS; nws >= 2; --nws)
+    for (nxs = kMaxXS; nxs >= (nws == kMaxWS ? 4 : 3); --nxs)
+      if (fused_smem_bytes(nxs, nws, dgroup, P.L) <= (size_t)optin) return true;
   return false;
 }
 
 cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*) {
-  const size_t sm = fused_smem_bytes(Ps.f_nxs, Ps.f_dgroup);
+  const size_t sm = fused_smem_bytes(Ps.f_nxs, Ps.f_nws, Ps.f_dgroup, Ps.L);
   cudaError_t err = cudaFuncSetAttribute(layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (err != cudaSuccess) return err;
   layer_fused_kernel<<<grid, kFThreads, sm, st>>>(Ps);
@@ -823,7 +845,7 @@ cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*)
 // -> fused SO(2) layer; then the destinations that cross tile boundaries or have none.
 cudaError_t launch_layer_fused(const TcParams& P0, const TcWeights& W, cudaStream_t st) {
   TcParams P = P0;
-  if (!fused_layout(P, P.f_nxs, P.f_dgroup)) return cudaErrorInvalidValue;
+  if (!fused_layout(P, P.f_nxs, P.f_nws, P.f_dgroup)) return cudaErrorInvalidValue;
   if (P.n_edges > 0) edge_dst_kernel<<<(P.n_atoms * 32 + 255) / 256, 256, 0, st>>>(P.row_ptr, P.n_atoms, P.edge_dst);
   cudaError_t err = launch_tc_pipeline(P, W, st, fused_consumer, nullptr, true);
   if (err != cudaSuccess) return err;

@@ -68,7 +68,7 @@ struct TcParams {
   float* slots;
   int rec_floats;
   int own_b;                     // bit l set: the fused layer's second epilogue group owns degree l
-  int f_nxs, f_dgroup;           // fused layer: x stages, floats of its work buffer per epilogue group
+  int f_nxs, f_nws, f_dgroup;    // fused layer: x and weight stages, floats of its work buffer per group
   int npass;
   TcPass pass[32];
   int woff[8];

@@ -635,12 +635,16 @@ __global__ void __launch_bounds__(kGRThreads, 1) gate_rotate_kernel(const __grid
         int sv = 0, dv = 0;
         if (e < E) {
           sv = P.src[e];
-          int lo = 0, hi = P.n_atoms;
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+          if (P.edge_dst) {   // layer calls: the destination of every edge is precomputed
+            dv = P.edge_dst[e];
+          } else {
+            int lo = 0, hi = P.n_atoms;
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (P.row_ptr[mid] <= e) lo = mid; else hi = mid;
+            }
+            dv = lo;
           }
-          dv = lo;
           if (sv < 0 || sv >= P.n_atoms) {
             egnn_flag(P.status, EGNN_DEV_INDEX_RANGE);
             sv = dv;

@@ -65,11 +65,12 @@ def layer_flops_per_edge(w) -> float:
     return 2.0 * macs
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_traffic_gst_8064.json")
+TRAFFIC_WORKLOAD = "hfo2_3000"   # the layer call whose DRAM counters are committed (scaled by edges)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", f"layer_traffic_{TRAFFIC_WORKLOAD}.json")
 TRAFFIC_SOURCES = ["equivariant_gnn_electronic_b200/csrc/so2_fused.cu", "equivariant_gnn_electronic_b200/csrc/so2_tc.cu",
                    "equivariant_gnn_electronic_b200/csrc/so2_tc.cuh", "equivariant_gnn_electronic_b200/csrc/tc_ptx.cuh",
                    "equivariant_gnn_electronic_b200/csrc/api.cu"]
-LAYER_KERNELS = ("prep_weights", "gate_kernel", "rotate_kernel", "layer_fused_kernel", "combine_kernel")
+LAYER_KERNELS = ("edge_dst_kernel", "prep_weights", "gate_rotate_kernel", "layer_fused_kernel", "combine_kernel")
 
 
 def sources_sha1() -> str:
@@ -101,7 +102,7 @@ def ingest_traffic(csv_path: str, workload: str, edges: int) -> None:
         v = float(r[vi].replace(",", ""))
         unit = r[ui].lower()
         scale = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "nsecond": 1e-6, "usecond": 1e-3,
-                 "msecond": 1.0}.get(unit, 1.0)
+                 "msecond": 1.0, "ns": 1e-6, "us": 1e-3, "ms": 1.0}.get(unit, 1.0)
         launches.setdefault((r[idi], name), {})[r[mi]] = v * scale
     per = {}
     for (_, name), m in launches.items():
@@ -114,7 +115,7 @@ def ingest_traffic(csv_path: str, workload: str, edges: int) -> None:
     rec = {"workload": workload, "edges": edges, "sources": TRAFFIC_SOURCES, "sources_sha1": sources_sha1(),
            "kernels": list(per.values()), "bytes_per_edge": tot * 1e9 / edges,
            "note": "one ncu capture of one layer call; counters from a single pass per launch"}
-    json.dump(rec, open(TRAFFIC_FILE, "w"), indent=1)
+    json.dump(rec, open(os.path.join(ROOT, "profiles", f"layer_traffic_{workload}.json"), "w"), indent=1)
     print(json.dumps(rec, indent=1))
 
 

@@ -387,6 +387,9 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
   if (warp == 0) {
     // ---------------- bulk copies: weight tiles and the rotate kernel's x tiles ----------------
     if (lane == 0) {
+      // x tiles stay in L2 until the last pass of their |m| block reads them; the weight
+      // image is read by every CTA and stays too
+      const uint64_t keep = tc::policy_evict_last(), drop = tc::policy_evict_first();
       uint32_t ix = 0, iw = 0;
       for (int t = P.t_begin + blockIdx.x; t < P.t_end && !*abort; t += gridDim.x) {
         const uint8_t* xt = P.X + (long long)(t - P.t_begin) * P.nch * 16384;
@@ -394,19 +397,21 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           const TcPass& ps = P.pass[p];
           const uint32_t bytes = (uint32_t)ps.n * 128u;
           const int nx = ps.block > 0 ? 2 : 1;
+          const bool last_of_block = p + 1 == P.npass || P.pass[p + 1].block != ps.block;
+          const uint64_t xpol = last_of_block ? drop : keep;
           for (int kb = 0; kb < ps.nk && !*abort; ++kb, ++iw) {
             const int sw = iw % nws;
             if (!tc::mbar_wait(tc::smem_u32(&ctl->w_empty[sw]), ((iw / nws) & 1) ^ 1, P.status, abort, 64)) break;
             tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->w_full[sw]), bytes);
-            tc::bulk_g2s(W_u32 + sw * kWBytes, P.wprep + ps.boff + (long long)kb * bytes, bytes,
-                         tc::smem_u32(&ctl->w_full[sw]));
+            tc::bulk_g2s_hint(W_u32 + sw * kWBytes, P.wprep + ps.boff + (long long)kb * bytes, bytes,
+                              tc::smem_u32(&ctl->w_full[sw]), keep);
             for (int h = 0; h < nx; ++h, ++ix) {
               const int sx = ix % nxs;
               if (!tc::mbar_wait(tc::smem_u32(&ctl->x_empty[sx]), ((ix / nxs) & 1) ^ 1, P.status, abort, 64)) break;
               const int id = ps.block == 0 ? kb : P.xbase[ps.block] + 2 * kb + h;
               tc::mbar_arrive_expect_tx(tc::smem_u32(&ctl->x_full[sx]), (uint32_t)kXBytes);
-              tc::bulk_g2s(X_u32 + sx * kXBytes, xt + (long long)id * kXBytes, (uint32_t)kXBytes,
-                           tc::smem_u32(&ctl->x_full[sx]));
+              tc::bulk_g2s_hint(X_u32 + sx * kXBytes, xt + (long long)id * kXBytes, (uint32_t)kXBytes,
+                                tc::smem_u32(&ctl->x_full[sx]), xpol);
             }
           }
         }

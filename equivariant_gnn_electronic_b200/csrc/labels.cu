@@ -14,9 +14,9 @@
 // Kernels:
 //   apply_terms       both directions: groups of blocks (or label vectors) brought into
 //                     shared memory by 1-D bulk copies, the next group's copy in flight
-//                     while the current one is summed; one (item, output element) per
-//                     work item summing its precomputed Clebsch-Gordan terms; the term
-//                     lists are built on the host from the orbital template.
+//                     while the current one is summed; one output element over a run
+//                     of items per work slot, summing its precomputed Clebsch-Gordan
+//                     terms; the term lists are built on the host from the template.
 //   h_count / h_scan / h_fill  block-sparse rows of the k = 0 Hamiltonian: row block d
 //                     holds the on-site block of d and, per distinct source atom s of
 //                     d's incoming edges, the sum of those edges' blocks (periodic
@@ -133,9 +133,11 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
 // group's inputs are contiguous in global memory and arrive by one 1-D bulk copy into
 // one of two shared-memory stages, issued one group ahead; a group whose byte count is
 // not a multiple of 16 (only a ragged last group can be) is loaded by all threads
-// instead.  One (item, q) output per work item: consecutive work items are consecutive
-// outputs of the group, so the stores are contiguous.  Waits are bounded (2 s); a wait
+// instead.  A work slot is one output q over a run of up to kRun items: q's terms are
+// read once and applied to the run's items in registers; consecutive slots are
+// consecutive outputs, so the stores are contiguous.  Waits are bounded (2 s); a wait
 // that runs out ends every thread's loop at the same group.
+constexpr int kRun = 16;   // items of a work slot
 __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restrict__ in, int nin, long long n,
                                                           const int* __restrict__ ptr, const int2* __restrict__ term,
                                                           int nout, int nterm, int staged, int te, int bulk,
@@ -200,19 +202,29 @@ __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restric
       for (int i = tid; i < ne * nin; i += nt) In[i] = in[g0 * nin + i];
       __syncthreads();
     }
-    int e = tid / nout, q = tid - e * nout;
+    // work slot = (output q, run of up to kRun items): the output's terms are read once
+    // and applied to the run's items held in registers; consecutive slots are
+    // consecutive outputs, so each store instruction covers consecutive addresses
+    const int nrun = (ne + kRun - 1) / kRun;
     float* o = out + g0 * nout;
-    for (int w = tid; w < ne * nout; w += nt) {
-      const float* x = In + e * nin;
+    for (int sl = tid; sl < nout * nrun; sl += nt) {
+      const int r = sl / nout, q = sl - r * nout;
+      const int e0 = r * kRun, m = ne - e0 < kRun ? ne - e0 : kRun;
+      float v[kRun];
+#pragma unroll
+      for (int i = 0; i < kRun; ++i) v[i] = 0.f;
       const int t1 = s_ptr[q + 1];
-      float v = 0.f;
       for (int t = s_ptr[q]; t < t1; ++t) {
         const int2 tm = s_term[t];
-        v = fmaf(__int_as_float(tm.y), x[tm.x], v);
+        const float cf = __int_as_float(tm.y);
+        const float* x = In + e0 * nin + tm.x;
+#pragma unroll
+        for (int i = 0; i < kRun; ++i)
+          if (i < m) v[i] = fmaf(cf, x[i * nin], v[i]);
       }
-      o[w] = v;
-      q += nt;
-      while (q >= nout) { q -= nout; ++e; }
+#pragma unroll
+      for (int i = 0; i < kRun; ++i)
+        if (i < m) o[(size_t)(e0 + i) * nout + q] = v[i];
     }
     __syncthreads();   // stage st is free for the copy issued in the next iteration
   }

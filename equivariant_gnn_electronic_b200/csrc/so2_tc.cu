@@ -279,6 +279,8 @@ __global__ void __launch_bounds__(128) head_blocks_kernel(const __grid_constant_
   }
 }
 
+constexpr int kHRun = 8;   // edges of a head_label work slot
+
 // 32-bit words of the staged tables of head_label_kernel, each region rounded up to a
 // multiple of four words (16 bytes); zero when the tables are read from global memory.
 struct HeadTabWords {
@@ -305,8 +307,9 @@ __host__ __device__ inline HeadTabWords head_tab_words(int n_lab, int n_entries,
 // group whose Wigner bytes are not a multiple of 16 is loaded by all threads); every
 // label from its precomputed list of (Wigner offset, record offset) pairs; every block
 // entry from its precomputed list of (label, Clebsch-Gordan coefficient) terms (both
-// built on the host from the orbital template and the pass layout).  Work items are
-// (edge, label) and (edge, entry) pairs, so the block stores are contiguous.
+// built on the host from the orbital template and the pass layout).  A work slot is one
+// label (or block entry) over a run of kHRun edges, so its term list is read once per
+// run and the block stores are contiguous.
 __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__ TcParams P,
                                                          const __grid_constant__ HeadLabelTabs Tb,
                                                          float* __restrict__ blocks, int te, int staged, int bulk) {
@@ -389,38 +392,51 @@ __global__ void __launch_bounds__(256) head_label_kernel(const __grid_constant__
       for (int i = tid; i < ne * wfl; i += nt) Ds[i] = P.wig[e0 * wfl + i];
       __syncthreads();
     }
-    // labels, one (edge, label) per work item: Ls[e][q] is item e * nlab + q
-    {
-      int e = tid / nlab, q = tid - e * nlab;
-      for (int w = tid; w < ne * nlab; w += nt) {
-        const int* lt = s_lab + q * 11;
-        const int cnt = lt[0];
-        const float* De = Ds + e * wfl;
-        const float* Re = Rs + e * nrec;
-        float h = 0.f;
-        for (int j = 0; j < cnt; ++j) h = fmaf(De[lt[1 + j]], Re[lt[6 + j]], h);
-        Ls[w] = h;
-        q += nt;
-        while (q >= nlab) { q -= nlab; ++e; }
+    // labels: work slot = (label q, run of up to kHRun edges); q's (Wigner, record)
+    // offsets are read once per slot
+    const int nrun = (ne + kHRun - 1) / kHRun;
+    for (int sl = tid; sl < nlab * nrun; sl += nt) {
+      const int r = sl / nlab, q = sl - r * nlab;
+      const int e0r = r * kHRun, m = ne - e0r < kHRun ? ne - e0r : kHRun;
+      const int* lt = s_lab + q * 11;
+      const int cnt = lt[0];
+      float h[kHRun];
+#pragma unroll
+      for (int i = 0; i < kHRun; ++i) h[i] = 0.f;
+      for (int j = 0; j < cnt; ++j) {
+        const float* De = Ds + e0r * wfl + lt[1 + j];
+        const float* Re = Rs + e0r * nrec + lt[6 + j];
+#pragma unroll
+        for (int i = 0; i < kHRun; ++i)
+          if (i < m) h[i] = fmaf(De[i * wfl], Re[i * nrec], h[i]);
       }
+#pragma unroll
+      for (int i = 0; i < kHRun; ++i)
+        if (i < m) Ls[(e0r + i) * nlab + q] = h[i];
     }
     __syncthreads();
-    // block entries, one (edge, entry) per work item: consecutive items are consecutive
-    // entries of the group's output, so the stores are contiguous
+    // block entries: work slot = (entry q, run of edges); consecutive slots are
+    // consecutive entries, so each store instruction covers consecutive addresses
     {
-      int e = tid / nb, q = tid - e * nb;
       float* out = blocks + e0 * nb;
-      for (int w = tid; w < ne * nb; w += nt) {
-        const float* Le = Ls + e * nlab;
+      for (int sl = tid; sl < nb * nrun; sl += nt) {
+        const int r = sl / nb, q = sl - r * nb;
+        const int e0r = r * kHRun, m = ne - e0r < kHRun ? ne - e0r : kHRun;
+        float v[kHRun];
+#pragma unroll
+        for (int i = 0; i < kHRun; ++i) v[i] = 0.f;
         const int t1 = s_tptr[q + 1];
-        float v = 0.f;
         for (int t = s_tptr[q]; t < t1; ++t) {
           const int2 tm = s_term[t];
-          v = fmaf(__int_as_float(tm.y), Le[tm.x], v);
+          const float cf = __int_as_float(tm.y);
+          const float* Le = Ls + e0r * nlab + tm.x;
+#pragma unroll
+          for (int i = 0; i < kHRun; ++i)
+            if (i < m) v[i] = fmaf(cf, Le[i * nlab], v[i]);
         }
-        out[w] = v;
-        q += nt;
-        while (q >= nb) { q -= nb; ++e; }
+#pragma unroll
+        for (int i = 0; i < kHRun; ++i)
+          if (i < m) out[(size_t)(e0r + i) * nb + q] = v[i];
       }
     }
     __syncthreads();   // stage st and Ls are free for the next iteration

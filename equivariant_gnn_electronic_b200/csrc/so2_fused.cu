@@ -340,6 +340,8 @@ __device__ __noinline__ void m0_logits(const __nv_bfloat16* Amat, int C, int H, 
   }
 }
 
+// LM = lmax: the degree switches below only instantiate the helpers a launch can reach.
+template <int LM>
 __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = tc::smem_u32(smem_raw);
@@ -632,13 +634,13 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
         for (int q2 = 0; q2 < l; ++q2) offz += pad4(2 * q2 + 1);
         const uint4* st_row = reinterpret_cast<const uint4*>(stash + ((size_t)l * C + c) * 128);
         switch (l) {
-          case 0: y0_degree<1>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          case 1: y0_degree<3>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          case 2: y0_degree<5>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          case 3: y0_degree<7>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          case 4: y0_degree<9>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          case 5: y0_degree<11>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
-          default: y0_degree<13>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 0: y0_degree<(LM >= 0 ? 1 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 1: y0_degree<(LM >= 1 ? 3 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 2: y0_degree<(LM >= 2 ? 5 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 3: y0_degree<(LM >= 3 ? 7 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 4: y0_degree<(LM >= 4 ? 9 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          case 5: y0_degree<(LM >= 5 ? 11 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
+          default: y0_degree<(LM >= 6 ? 13 : 2 * LM + 1)>(EA, es, m0r, t, l, c, hh, nvalid, DZ, offz, st_row); break;
         }
       };
       unsigned y0_left = 0;
@@ -685,12 +687,12 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
           tc::tc_fence_after();
           const uint32_t tb = tl + buf * 256;
           switch (l) {
-            case 1: pm_degree<3>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 2: pm_degree<5>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 3: pm_degree<7>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 4: pm_degree<9>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
-            case 5: pm_degree<11>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
-            default: pm_degree<13>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 1: pm_degree<(LM >= 1 ? 3 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 2: pm_degree<(LM >= 2 ? 5 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 3: pm_degree<(LM >= 3 ? 7 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 4: pm_degree<(LM >= 4 ? 9 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            case 5: pm_degree<(LM >= 5 ? 11 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
+            default: pm_degree<(LM >= 6 ? 13 : 2 * LM + 1)>(EA, es, dcur, t, l, c, hh, nvalid, tb); break;
           }
           tc::tc_fence_before();
           tc::mbar_arrive(tc::smem_u32(&ctl->acc_empty[buf]));
@@ -838,9 +840,19 @@ bool fused_layout(const TcParams& P, int& nxs, int& nws, int& dgroup) {
 
 cudaError_t fused_consumer(const TcParams& Ps, int grid, cudaStream_t st, void*) {
   const size_t sm = fused_smem_bytes(Ps.f_nxs, Ps.f_nws, Ps.f_dgroup, Ps.L);
-  cudaError_t err = cudaFuncSetAttribute(layer_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (err != cudaSuccess) return err;
-  layer_fused_kernel<<<grid, kFThreads, sm, st>>>(Ps);
+  cudaError_t err = cudaSuccess;
+  switch (Ps.lmax) {
+#define EGNN_FUSED_CASE(LMv)                                                                             \
+  case LMv:                                                                                              \
+    err = cudaFuncSetAttribute(layer_fused_kernel<LMv>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+    if (err != cudaSuccess) return err;                                                                  \
+    layer_fused_kernel<LMv><<<grid, kFThreads, sm, st>>>(Ps);                                           \
+    break;
+    EGNN_FUSED_CASE(1) EGNN_FUSED_CASE(2) EGNN_FUSED_CASE(3) EGNN_FUSED_CASE(4) EGNN_FUSED_CASE(5) EGNN_FUSED_CASE(6)
+#undef EGNN_FUSED_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -759,7 +759,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layer_fused_kernel(const __grid_
 // their embedding; atoms whose edges cross tile boundaries merge their per-tile
 // records (softmax maxima and sums rescaled to the common maximum).  One CTA of C
 // threads (thread = channel) per atom.
-__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(128, 8) combine_kernel(const __grid_constant__ TcParams P) {
   const int d = blockIdx.x, c = threadIdx.x;
   const int C = P.C, L2 = P.L2, hh = c / (C / P.H);
   const size_t o = (size_t)d * L2 * C + c;
@@ -771,29 +771,33 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Tc
   const int t0 = b >> 7, t1 = (en - 1) >> 7;
   if (t0 == t1) return;
   const size_t rf = P.rec_floats;
+  auto record = [&](int t) { return P.slots + ((size_t)t * 2 + (t == t0 ? 1 : 0)) * rf; };
   float mx = -INFINITY;
-  for (int t = t0; t <= t1; ++t) {
-    const float* rec = P.slots + ((size_t)t * 2 + (t == t0 ? 1 : 0)) * rf + (size_t)L2 * C;
-    mx = fmaxf(mx, rec[hh]);
-  }
-  float acc[49];
-#pragma unroll
-  for (int i = 0; i < 49; ++i) acc[i] = 0.f;
+  for (int t = t0; t <= t1; ++t) mx = fmaxf(mx, record(t)[(size_t)L2 * C + hh]);
   float sum = 0.f;
   for (int t = t0; t <= t1; ++t) {
-    const float* rec = P.slots + ((size_t)t * 2 + (t == t0 ? 1 : 0)) * rf;
-    const float w = __expf(rec[(size_t)L2 * C + hh] - mx);
-    sum += w * rec[(size_t)L2 * C + 16 + hh];
-#pragma unroll
-    for (int i = 0; i < 49; ++i)
-      if (i < L2) acc[i] += w * rec[(size_t)i * C + c];
+    const float* rec = record(t) + (size_t)L2 * C;
+    sum += __expf(rec[hh] - mx) * rec[16 + hh];
   }
   const float inv = 1.0f / sum;
+  // rows in chunks of 8: few registers, so many atoms are in flight per SM
+  for (int i0 = 0; i0 < L2; i0 += 8) {
+    float acc[8];
 #pragma unroll
-  for (int i = 0; i < 49; ++i)
-    if (i < L2)
-      P.node_out[o + (size_t)i * C] =
-          __float2bfloat16_rn(__bfloat162float(P.node_in[o + (size_t)i * C]) + acc[i] * inv);
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int t = t0; t <= t1; ++t) {
+      const float* rec = record(t);
+      const float w = __expf(rec[(size_t)L2 * C + hh] - mx);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i0 + i < L2) acc[i] += w * rec[(size_t)(i0 + i) * C + c];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i0 + i < L2)
+        P.node_out[o + (size_t)(i0 + i) * C] =
+            __float2bfloat16_rn(__bfloat162float(P.node_in[o + (size_t)(i0 + i) * C]) + acc[i] * inv);
+  }
 }
 
 // Destination atom of every edge (one warp per atom; consecutive edges, coalesced stores).

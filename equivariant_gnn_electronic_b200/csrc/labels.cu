@@ -74,7 +74,10 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
   }
   T.n_lab = lab;
   const int norb = o, nb = norb * norb;
-  // (label, entry, coefficient) of every Clebsch-Gordan term of a block
+  // (label, entry, coefficient) of every nonzero Clebsch-Gordan term of a block: the
+  // real coupling matrices are sparse (431 of 2,025 coefficients are nonzero for the
+  // {s,s,p,p,d} template), and the smallest nonzero one for l <= 3 is far above the
+  // round-off left where the complex-to-real sums cancel exactly
   std::vector<int> t_lab, t_ent;
   std::vector<float> t_cg;
   for (int a = 0; a < n_shells; ++a)
@@ -87,9 +90,11 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
         for (int ia = 0; ia < 2 * la + 1; ++ia)
           for (int jb = 0; jb < 2 * lb + 1; ++jb)
             for (int M = 0; M < 2 * L + 1; ++M) {
+              const float c = cg[(ia * (2 * lb + 1) + jb) * (2 * L + 1) + M];
+              if (fabsf(c) < 1e-6f) continue;
               t_lab.push_back(lab_off[L] + M * mult[L] + k);
               t_ent.push_back((shell_off[a] + ia) * norb + shell_off[b] + jb);
-              t_cg.push_back(cg[(ia * (2 * lb + 1) + jb) * (2 * L + 1) + M]);
+              t_cg.push_back(c);
             }
       }
     }

@@ -16,7 +16,8 @@
 //                     shared memory by 1-D bulk copies, the next group's copy in flight
 //                     while the current one is summed; one output element over a run
 //                     of items per work slot, summing its precomputed Clebsch-Gordan
-//                     terms; the term lists are built on the host from the template.
+//                     terms; the term lists are built on the host from the template,
+//                     once per template.
 //   h_count / h_scan / h_fill  block-sparse rows of the k = 0 Hamiltonian: row block d
 //                     holds the on-site block of d and, per distinct source atom s of
 //                     d's incoming edges, the sum of those edges' blocks (periodic
@@ -24,6 +25,9 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
+#include <memory>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -42,13 +46,16 @@ struct LabelTables {
   const int2* l_term;     // ... (block entry index, coefficient as float bits)
 };
 
-// Builds the template's term lists on the host and copies them into `ws` (asynchronous
-// copies on `st` from pageable host memory, staged before the call returns).
-egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T, void* ws, size_t ws_bytes,
-                        cudaStream_t st) {
-  if (!shell_l || n_shells < 1 || n_shells > 16) return EGNN_ERR_INVALID_ARG;
-  memset(&T, 0, sizeof(T));
-  T.n_shells = n_shells;
+// A template's term lists on the host: built once per template, then kept.
+struct HostTables {
+  std::vector<int32_t> shells;
+  int n_orb = 0, n_lab = 0, lmax = 0;
+  std::vector<int> bptr, lptr;       // [n_orb^2 + 1], [n_lab + 1]
+  std::vector<int2> bterm, lterm;    // [n_term] each
+};
+
+// Builds the term lists of the template shell_l[0 .. n_shells).
+egnn_status build_host_tables(const int32_t* shell_l, int32_t n_shells, HostTables& H) {
   int o = 0, lmax = 0, shell_off[17];
   for (int a = 0; a < n_shells; ++a) {
     const int l = shell_l[a];
@@ -58,8 +65,9 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
     o += 2 * l + 1;
     lmax = 2 * l > lmax ? 2 * l : lmax;
   }
-  T.n_orb = o;
-  T.lmax = lmax;
+  H.shells.assign(shell_l, shell_l + n_shells);
+  H.n_orb = o;
+  H.lmax = lmax;
   // label order: L, then M, then k over the pairs (a, b) containing L (a outer)
   int mult[8] = {0}, lab_off[8] = {0};
   std::vector<int> kidx(n_shells * n_shells * 8, 0);
@@ -72,7 +80,7 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
     lab_off[L] = lab;
     lab += (2 * L + 1) * mult[L];
   }
-  T.n_lab = lab;
+  H.n_lab = lab;
   const int norb = o, nb = norb * norb;
   // (label, entry, coefficient) of every nonzero Clebsch-Gordan term of a block: the
   // real coupling matrices are sparse (431 of 2,025 coefficients are nonzero for the
@@ -99,7 +107,6 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
       }
     }
   const int nt = (int)t_cg.size();
-  T.n_term = nt;
   // CSR by entry and by label (stable order: the sums run in a fixed order)
   std::vector<int> bptr(nb + 1, 0), lptr(lab + 1, 0);
   for (int i = 0; i < nt; ++i) {
@@ -118,14 +125,59 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
     x.x = t_ent[i];
     lterm[lfill[t_lab[i]]++] = x;
   }
+  H.bptr = std::move(bptr);
+  H.lptr = std::move(lptr);
+  H.bterm = std::move(bterm);
+  H.lterm = std::move(lterm);
+  return EGNN_OK;
+}
+
+// Templates whose term lists were built, most recent last (at most kTabCache).  Building
+// one takes about a millisecond of host time (the Clebsch-Gordan coefficients from the
+// Racah formula), longer than a conversion of a 100k-orbital structure on the GPU.
+constexpr size_t kTabCache = 16;
+std::mutex g_tab_mu;
+std::vector<std::shared_ptr<const HostTables>> g_tab_cache;
+
+// Copies the template's term lists into `ws` (asynchronous copies on `st` from pageable
+// host memory, staged before the call returns), building them on the first call for the
+// template.  An invalid template is rejected on every call and never kept.
+egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
+  if (!shell_l || n_shells < 1 || n_shells > 16) return EGNN_ERR_INVALID_ARG;
+  std::shared_ptr<const HostTables> H;
+  {
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    for (const auto& c : g_tab_cache)
+      if ((int)c->shells.size() == n_shells && std::equal(c->shells.begin(), c->shells.end(), shell_l)) {
+        H = c;
+        break;
+      }
+  }
+  if (!H) {
+    auto h = std::make_shared<HostTables>();
+    const egnn_status s = build_host_tables(shell_l, n_shells, *h);
+    if (s != EGNN_OK) return s;
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    if (g_tab_cache.size() >= kTabCache) g_tab_cache.erase(g_tab_cache.begin());
+    g_tab_cache.push_back(h);
+    H = h;
+  }
+  memset(&T, 0, sizeof(T));
+  T.n_shells = n_shells;
+  T.n_orb = H->n_orb;
+  T.n_lab = H->n_lab;
+  T.lmax = H->lmax;
+  T.n_term = (int)H->bterm.size();
+  const int nb = H->n_orb * H->n_orb, lab = H->n_lab, nt = T.n_term;
   const size_t o1 = ((nb + 1) * 4 + 15) & ~(size_t)15, o2 = o1 + (size_t)nt * 8;
   const size_t o3 = o2 + (((lab + 1) * 4 + 15) & ~(size_t)15), need = o3 + (size_t)nt * 8;
   if (!ws || ws_bytes < need) return EGNN_ERR_INVALID_ARG;
   char* w = (char*)ws;
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w, bptr.data(), (nb + 1) * 4, cudaMemcpyHostToDevice, st));
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o1, bterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o2, lptr.data(), (lab + 1) * 4, cudaMemcpyHostToDevice, st));
-  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o3, lterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w, H->bptr.data(), (nb + 1) * 4, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o1, H->bterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o2, H->lptr.data(), (lab + 1) * 4, cudaMemcpyHostToDevice, st));
+  EGNN_CUDA_TRY(cudaMemcpyAsync(w + o3, H->lterm.data(), (size_t)nt * 8, cudaMemcpyHostToDevice, st));
   T.b_ptr = (const int*)w;
   T.b_term = (const int2*)(w + o1);
   T.l_ptr = (const int*)(w + o2);
@@ -358,25 +410,62 @@ __global__ void __launch_bounds__(256) h_fill_kernel(const int32_t* __restrict__
   int n_lo = 0;
   for (int k = 0; k < nrun; ++k) n_lo += run_s[k] < d ? 1 : 0;
   const int row0 = bsr_row_ptr[d], nblk = bsr_row_ptr[d + 1] - row0;
-  for (int j = 0; j < nblk; ++j) {
-    int k = -1;   // run of block j (-1: on-site only)
-    int col = d;
+  // run k of block j (-1: on-site only) and its column
+  auto block_of = [&](int j, int& k, int& col) {
     if (j < n_lo) {
       k = j;
       col = run_s[k];
     } else if (j == n_lo) {
       k = self_run;
+      col = d;
     } else {
       k = j - 1 + (self_run >= 0 ? 1 : 0);
       col = run_s[k];
     }
-    if (tid == 0) bsr_col[row0 + j] = col;
-    float* out = bsr_val + (size_t)(row0 + j) * nb;
-    for (int q = tid; q < nb; q += blockDim.x) {
-      float v = col == d ? onsite[(size_t)d * nb + q] : 0.f;
-      if (k >= 0)
-        for (int e = run_b[k]; e < run_b[k + 1]; ++e) v += edge_blocks[(size_t)e * nb + q];
-      out[q] = v;
+  };
+  for (int j = tid; j < nblk; j += blockDim.x) {
+    int k, col;
+    block_of(j, k, col);
+    bsr_col[row0 + j] = col;
+  }
+  // all nblk * nb output elements of the row block (contiguous in bsr_val), kU per
+  // thread per pass: the on-site term and the first edge of all kU elements are loaded
+  // before any is summed, so kU loads per thread are in flight (a run is mostly one
+  // edge).  Each element sums on-site, then its run's edges in edge order.
+  constexpr int kU = 4;
+  const int tot = nblk * nb;
+  float* out = bsr_val + (size_t)row0 * nb;
+  for (int i0 = tid; i0 < tot; i0 += kU * blockDim.x) {
+    float a[kU], v[kU];
+    int kk[kU], qq[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      a[u] = 0.f;
+      v[u] = 0.f;
+      kk[u] = -1;
+      qq[u] = 0;
+      if (i < tot) {
+        const int j = i / nb, q = i - j * nb;
+        int k, col;
+        block_of(j, k, col);
+        kk[u] = k;
+        qq[u] = q;
+        if (col == d) a[u] = onsite[(size_t)d * nb + q];
+        if (k >= 0) v[u] = edge_blocks[(size_t)run_b[k] * nb + q];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      if (i >= tot) continue;
+      const int k = kk[u];
+      float x = a[u];
+      if (k >= 0) {
+        x += v[u];
+        for (int e = run_b[k] + 1; e < run_b[k + 1]; ++e) x += edge_blocks[(size_t)e * nb + qq[u]];
+      }
+      out[i] = x;
     }
   }
 }

@@ -194,7 +194,11 @@ egnn_status make_tables(const int32_t* shell_l, int32_t n_shells, LabelTables& T
 // read once and applied to the run's items in registers; consecutive slots are
 // consecutive outputs, so the stores are contiguous.  Waits are bounded (2 s); a wait
 // that runs out ends every thread's loop at the same group.
-constexpr int kRun = 16;   // items of a work slot
+// Items of a work slot.  A group of 32 items makes three runs (11, 11, 10), so the 169
+// outputs of a 13-orbital template give 507 slots: two nearly full passes of 256 threads
+// (runs of 16 gave 338 slots, the second pass a third full; runs of 8 cost more term
+// reads per item than the fuller passes saved).
+constexpr int kRun = 11;
 __global__ void __launch_bounds__(256) apply_terms_kernel(const float* __restrict__ in, int nin, long long n,
                                                           const int* __restrict__ ptr, const int2* __restrict__ term,
                                                           int nout, int nterm, int staged, int te, int bulk,
